@@ -1,0 +1,276 @@
+"""Pins for the CPU oracle, checked against what the pages and the mathematics fix.
+
+Each test compares the oracle with something other than itself: the worked
+memory figure printed in the RIPE abstract, closed forms, textbook attention
+computed by a library routine (torch scaled_dot_product_attention in fp64),
+an independent brute-force formulation, and the block-independence property
+the abstract states.  Runs on CPU only.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ripe_oracle as orc
+from self_speculative_decode_b200.synth import PlaneSource, block_from_planes
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f64(bits):
+    # local widening of bf16 bits, independent of the oracle's helper
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def _cache(N, kvH, g, d, R, W, T, B, rho=0.88, seed=0, mode=orc.QUERY_RELATIVE, independent=False):
+    src = PlaneSource(N, kvH, d, R, T + B, rho, seed, independent=independent)
+    PK = [src.plane(r, "K") for r in range(R)]
+    PV = [src.plane(r, "V") for r in range(R)]
+    c = orc.OracleCache(N, 1, kvH, d, R, W, T + B, mode)
+    for pl in range(R):
+        c.load_prefix(0, pl, [T] * N, PK[pl], PV[pl])
+    for r in range(R):
+        c.append(0, r, block_from_planes(PK[r], T, B), block_from_planes(PV[r], T, B))
+    return c, PK, PV, src
+
+
+def _sdpa(q, K, V, T, B, g, scale):
+    """Textbook causal attention of block queries over keys [0, T+B) (torch, fp64)."""
+    Hq = q.shape[1]
+    qt = torch.from_numpy(q).permute(1, 0, 2).unsqueeze(0)               # [1, Hq, B, d]
+    kt = torch.from_numpy(K).repeat_interleave(g, dim=0).unsqueeze(0)   # [1, Hq, T+B, d]
+    vt = torch.from_numpy(V).repeat_interleave(g, dim=0).unsqueeze(0)
+    j = torch.arange(B)[:, None]
+    t = torch.arange(T + B)[None, :]
+    mask = t <= T + j
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale)
+    assert o.shape == (1, Hq, B, q.shape[2])
+    return o[0].permute(1, 0, 2).numpy()
+
+
+# ---------------------------------------------------------------- P1: memory
+def test_memory_fraction_matches_printed_worked_example():
+    vals = {}
+    with open(os.path.join(GOLDEN, "huginn_memory_fraction.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.strip().split("=")
+                vals[k] = float(v)
+    frac, stored = orc.memory_fraction(int(vals["T"]), int(vals["W"]), int(vals["R"]),
+                                       int(vals["recurrent_layers"]), int(vals["other_layers"]))
+    assert round(100 * frac, 1) == vals["printed_percent"]
+    # dropping the window planes (or counting W-1 of them) misses the printed figure
+    frac_short, _ = orc.memory_fraction(int(vals["T"]), int(vals["W"]) - 1, int(vals["R"]), 4, 4)
+    assert round(100 * frac_short, 1) != vals["printed_percent"]
+
+
+@pytest.mark.parametrize("T,W,R", [(1, 0, 3), (10, 3, 4), (7, 20, 5), (40, 8, 1), (33, 33, 2)])
+def test_stored_count_closed_form(T, W, R):
+    """Deepest plane everywhere + all R planes in the last W positions: T + min(W, T) * (R - 1)."""
+    frac, stored = orc.memory_fraction(T, W, R)
+    assert stored == T + min(W, T) * (R - 1)
+    assert abs(frac - (T + min(W, T) * (R - 1)) / (R * T)) < 1e-15
+
+
+def test_stored_count_independent_of_block_history():
+    rng = np.random.default_rng(5)
+    R, W = 4, 6
+    c = orc.OracleCache(N=2, L=2, kvH=1, d=2, R=R, W=W, max_T=200)
+    for _ in range(40):
+        B = int(rng.integers(1, 7))
+        blk = np.ones((2, B, 1, 2), dtype=np.uint16)
+        for layer in range(2):
+            for r in range(R):
+                c.append(layer, r, blk, blk)
+        c.commit(rng.integers(0, B + 1, size=2))
+        for n in range(2):
+            T = int(c.T[n])
+            for layer in range(2):
+                assert c.stored_position_planes(layer, n) == T + min(W, T) * (R - 1)
+
+
+# ---------------------------------------------------------------- P2 / P3 / P4
+@pytest.mark.parametrize("r", [0, 2, 3])
+def test_full_cache_is_textbook_attention_on_plane_r(r):
+    N, kvH, g, d, R, T, B = 1, 2, 2, 16, 4, 37, 5
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W=T + B, T=T, B=B, seed=1)
+    q = src.queries(r, B, kvH * g)
+    out, _ = c.verify(0, r, q, g, scale=0.7)
+    ref = _sdpa(_f64(q[0]), _f64(PK[r][0]), _f64(PV[r][0]), T, B, g, 0.7)
+    assert np.abs(out[0] - ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("r", [0, 1, 3])
+def test_window_zero_is_deepest_plane_prefix(r):
+    N, kvH, g, d, R, T, B = 1, 1, 3, 8, 4, 29, 6
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W=0, T=T, B=B, seed=2)
+    q = src.queries(r, B, kvH * g)
+    out, _ = c.verify(0, r, q, g)
+    K = np.concatenate([_f64(PK[R - 1][0])[:, :T], _f64(PK[r][0])[:, T:]], axis=1)
+    V = np.concatenate([_f64(PV[R - 1][0])[:, :T], _f64(PV[r][0])[:, T:]], axis=1)
+    ref = _sdpa(_f64(q[0]), K, V, T, B, g, 1.0)
+    assert np.abs(out[0] - ref).max() < 1e-12
+
+
+@pytest.mark.parametrize("W", [0, 3, 100])
+def test_single_loop_is_ordinary_attention(W):
+    N, kvH, g, d, T, B = 1, 2, 1, 8, 21, 4
+    c, PK, PV, src = _cache(N, kvH, g, d, R=1, W=W, T=T, B=B, seed=3)
+    q = src.queries(0, B, kvH * g)
+    out, _ = c.verify(0, 0, q, g)
+    ref = _sdpa(_f64(q[0]), _f64(PK[0][0]), _f64(PV[0][0]), T, B, g, 1.0)
+    assert np.abs(out[0] - ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------- P5
+def test_softmax_weights_sum_to_one():
+    N, kvH, g, d, R, W, T, B = 1, 1, 1, 8, 4, 5, 30, 4
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W, T, B, seed=4)
+    Kr, Vr, Kl, Vl, _ = c.verify_inputs(0, 1)
+    q = orc.bf16_to_f64(src.queries(1, B, 1))
+    for j in range(B):
+        for scale in (1.0, 8.0):
+            w = orc.weights(T, j, 1, R, W, Kr[0, 0], Kl[0, 0], q[0, j, 0], scale)
+            assert abs(w.sum() - 1.0) < 1e-12 and (w >= 0).all()
+    # with every value equal to one the output is exactly the weight sum
+    ones = np.ones_like(Vr)
+    out, _ = orc.verify(c.T, B, 1, R, W, g, Kr, np.where(np.isnan(Vr), np.nan, ones),
+                        Kl, np.where(np.isnan(Vl), np.nan, ones), q)
+    assert np.abs(out - 1.0).max() < 1e-12
+
+
+# ---------------------------------------------------------------- plane counts (closed form)
+def _count_closed_form(T, j, r, R, W, mode):
+    """Keys read at plane r by query p = T + j: [min(T, max(0, p - W)), p] (query window) or
+    [max(0, T - W), p] (cache window); the rest read plane R - 1."""
+    p = T + j
+    lo = min(T, max(0, p - W)) if mode == orc.QUERY_RELATIVE else max(0, T - W)
+    return p - lo + 1
+
+
+@pytest.mark.parametrize("mode", [orc.QUERY_RELATIVE, orc.CACHE_RELATIVE])
+@pytest.mark.parametrize("T,W,B,r", [(20, 4, 6, 1), (20, 0, 3, 0), (5, 9, 4, 2), (30, 6, 6, 3)])
+def test_plane_usage_counts(mode, T, W, B, r):
+    """Zero keys give uniform weights; one-hot values per plane reveal which planes were read."""
+    R, d = 4, 8
+    L = T + B
+    Kz = np.zeros((1, 1, L, d))
+    onehot = lambda pl: np.broadcast_to(np.eye(d)[pl], (1, 1, L, d)).copy()
+    out, _ = orc.verify([T], B, r, R, W, 1, Kz, onehot(r), Kz, onehot(R - 1), np.zeros((1, B, 1, d)),
+                        mode=mode)
+    for j in range(B):
+        p = T + j
+        n_r = _count_closed_form(T, j, r, R, W, mode)
+        if r == R - 1:
+            assert abs(out[0, j, 0, R - 1] - 1.0) < 1e-12
+        else:
+            assert abs(out[0, j, 0, r] * (p + 1) - n_r) < 1e-9
+            assert abs(out[0, j, 0, R - 1] * (p + 1) - (p + 1 - n_r)) < 1e-9
+
+
+def test_absent_plane_is_detected():
+    """Planes that RIPE does not store are NaN; asking for a wider window must fail loudly."""
+    N, kvH, g, d, R, W, T, B = 1, 1, 1, 8, 4, 3, 20, 2
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W, T, B, seed=6)
+    Kr, Vr, Kl, Vl, _ = c.verify_inputs(0, 0)
+    q = orc.bf16_to_f64(src.queries(0, B, 1))
+    orc.verify(c.T, B, 0, R, W, g, Kr, Vr, Kl, Vl, q)          # the cache's own window: fine
+    with pytest.raises(RuntimeError):
+        orc.verify(c.T, B, 0, R, W + 2, g, Kr, Vr, Kl, Vl, q)  # reads plane 0 outside the window
+
+
+# ---------------------------------------------------------------- P7 brute force
+@pytest.mark.parametrize("mode", [orc.QUERY_RELATIVE, orc.CACHE_RELATIVE])
+@pytest.mark.parametrize("T,W,B,r,g", [(12, 3, 4, 0, 2), (12, 0, 4, 2, 1), (6, 10, 3, 1, 3),
+                                       (15, 5, 6, 3, 1), (9, 1, 5, 1, 2)])
+def test_brute_force_twin(mode, T, W, B, r, g):
+    N, kvH, d, R = 1, 2, 8, 4
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W, T, B, seed=7, mode=mode, independent=True)
+    q = src.queries(r, B, kvH * g)
+    out, lse = c.verify(0, r, q, g, scale=1.3)
+    Kall = np.stack([_f64(PK[pl][0]) for pl in range(R)])
+    Vall = np.stack([_f64(PV[pl][0]) for pl in range(R)])
+    bo, bl = orc.brute_verify(Kall, Vall, T, B, r, W, g, _f64(q[0]), 1.3, mode)
+    assert np.abs(out[0] - bo).max() < 1e-12
+    assert np.abs(lse[0] - bl).max() < 1e-12
+    # planted mistake: an off-by-one window in the twin is visible at this size
+    if 0 < W < T and r != R - 1:
+        bo2, _ = orc.brute_verify(Kall, Vall, T, B, r, W + 1, g, _f64(q[0]), 1.3, mode)
+        assert np.abs(out[0] - bo2).max() > 1e-6
+
+
+# ---------------------------------------------------------------- P6 block independence
+def _decode(W, splits, mode, R=4, T0=10, S=12, kvH=1, g=2, d=8, seed=11):
+    """Verify positions T0..T0+S-1 in the given block split, committing every position.
+
+    Returns {(position, r): output row [Hq][d]} from the oracle state machine.
+    """
+    src = PlaneSource(1, kvH, d, R, T0 + S, 0.88, seed, independent=True)
+    PK = [src.plane(r, "K") for r in range(R)]
+    PV = [src.plane(r, "V") for r in range(R)]
+    qsrc = PlaneSource(1, kvH * g, d, R, T0 + S, 0.88, seed + 1000)
+    Q = [qsrc.plane(r, "K") for r in range(R)]           # per-position queries [1][Hq][pos][d]
+    c = orc.OracleCache(1, 1, kvH, d, R, W, T0 + S, mode)
+    for pl in range(R):
+        c.load_prefix(0, pl, [T0], PK[pl], PV[pl])
+    res = {}
+    t = T0
+    for B in splits:
+        for r in range(R):
+            c.append(0, r, block_from_planes(PK[r], t, B), block_from_planes(PV[r], t, B))
+        for r in range(R):
+            q = np.ascontiguousarray(Q[r][:, :, t:t + B].transpose(0, 2, 1, 3))
+            out, _ = c.verify(0, r, q, g)
+            for j in range(B):
+                res[(t + j, r)] = out[0, j]
+        c.commit([B])
+        t += B
+    assert t == T0 + 12
+    return res
+
+
+def _max_diff(a, b):
+    return max(np.abs(a[k] - b[k]).max() for k in a)
+
+
+@pytest.mark.parametrize("W", [4, 5, 9])
+def test_block_independence_when_window_covers_block(W):
+    B = 4
+    rng = np.random.default_rng(W)
+    ref = _decode(W, [1] * 12, orc.QUERY_RELATIVE)               # position by position
+    batched = _decode(W, [B] * 3, orc.QUERY_RELATIVE)            # blocks of B
+    splits = []
+    while sum(splits) < 12:
+        splits.append(int(min(rng.integers(1, W + 2), 12 - sum(splits))))
+    rand = _decode(W, splits, orc.QUERY_RELATIVE)                # random blocks of <= W+1
+    assert _max_diff(ref, batched) < 1e-12
+    assert _max_diff(ref, rand) < 1e-12
+
+
+def test_block_dependence_negative_controls():
+    # window shorter than the block: the batched result differs from the sequential one
+    assert _max_diff(_decode(1, [1] * 12, 0), _decode(1, [4] * 3, 0)) > 1e-3
+    # window measured from the cache end: differs even with W >= B
+    assert _max_diff(_decode(5, [1] * 12, orc.CACHE_RELATIVE),
+                     _decode(5, [4] * 3, orc.CACHE_RELATIVE)) > 1e-3
+
+
+# ---------------------------------------------------------------- state machine
+def test_rollback_discards_rejected_positions_and_evicts():
+    R, W = 3, 2
+    c = orc.OracleCache(N=1, L=1, kvH=1, d=1, R=R, W=W, max_T=20)
+    blk = lambda v, B: np.full((1, B, 1, 1), v, dtype=np.uint16)
+    for r in range(R):
+        c.append(0, r, blk(10 + r, 4), blk(20 + r, 4))
+    c.commit([3])                  # positions 0..2 kept, 3 discarded
+    assert int(c.T[0]) == 3
+    assert not c.present[0, :, 0, 3].any()
+    # window W=2 -> position 0 keeps only the deepest plane, 1 and 2 keep all
+    assert c.present[0, :, 0, 0].tolist() == [False, False, True]
+    assert c.present[0, :, 0, 1:3].all()
+    assert c.values(0, R - 1, "K")[0, 0, 0, 0] == 10 + R - 1
+    with pytest.raises(ValueError):
+        for r in range(R):
+            c.append(0, r, blk(1, 2), blk(1, 2))
+        c.commit([3])              # more than the block length
