@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Benchmark of the RIPE verification step on B200.
+
+A step is one verification pass of a draft block through every loop and recurrent layer
+(for r in 0..R-1, for layer in 0..L-1: append plane r of the block, verify at loop r),
+followed by the accept / rollback commit with window eviction -- every step of the hot
+path -- captured once as a CUDA graph and replayed.  Inputs are resident in HBM before the
+timed region; the per-step accepted lengths are drawn uniform on {0..B} from a seed.
+
+Default workload: Huginn-shaped verify (4 recurrent layers, 55 MHA heads x 96, R = 32,
+T = 1024, W = 64, B = 8, batch 1, planes approaching the deepest at 0.88 per loop).
+The same step is also timed with the full-cache and deepest-plane-only layouts.
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU (torchrun); every rank runs
+its own replica of the workload (independent sequences, no collective in the data path);
+times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "verify-attn GB/s (% of HBM peak) and verified tokens/s, RIPE vs full cache"
+FALLBACK_HBM_GBS = 6650.0
+
+CONFIGS = {
+    "huginn": dict(N=1, L=4, Hq=55, kvH=55, d=96, R=32, T=1024, W=64, B=8, rho=0.88,
+                   workload="Huginn-shaped verify: 4 recurrent layers, 55 MHA heads x 96, R=32, "
+                            "T=1024, W=64, B=8, batch 1, rho 0.88"),
+    "long_gqa": dict(N=8, L=4, Hq=32, kvH=8, d=128, R=32, T=32768, W=64, B=8, rho=0.85,
+                     workload="Long-context GQA: 4 recurrent layers, 32 q / 8 kv heads x 128, R=32, "
+                              "T=32768, W=64, B=8, batch 8, rho 0.85"),
+    "sweep": dict(N=4, L=1, Hq=55, kvH=55, d=96, R=32, T=4096, W=64, B=8, rho=0.81,
+                  workload="Window/block sweep point: 1 layer, 55 MHA heads x 96, R=32, T=4096, "
+                           "W=64, B=8, batch 4, rho 0.81"),
+    "tiny": dict(N=1, L=1, Hq=2, kvH=2, d=64, R=4, T=128, W=16, B=4, rho=0.88,
+                 workload="Tiny RIPE check: 1 layer, 2 heads x 64, R=4, T=128, W=16, B=4, batch 1"),
+}
+
+
+# ------------------------------------------------------------------ accounting
+def dual_keys(T, W, B, R, r, mode=0):
+    """Window keys read at the deepest plane by later queries of the block (query window)."""
+    if mode != 0 or r == R - 1:
+        return 0
+    D = max(0, T - W)
+    return max(0, min(T, T + B - 1 - W) - D)
+
+
+def verify_bytes(cfg, T_list, r):
+    """Algorithmic bytes of one verify call: one plane per key read (K and V), the extra
+    deepest-plane reads of the query window, the queries and the outputs."""
+    row = 4 * cfg["kvH"] * cfg["d"]               # K + V, bf16, all kv heads, one position
+    keys = sum(T + cfg["B"] + dual_keys(T, cfg["W"], cfg["B"], cfg["R"], r) for T in T_list)
+    qo = 2 * cfg["N"] * cfg["B"] * cfg["Hq"] * cfg["d"] * 2
+    return keys * row + qo
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def gpu_id(index):
+    """nvidia-smi identifier of a torch device (its UUID, robust to CUDA_VISIBLE_DEVICES)."""
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(index).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(index)
+
+
+# ------------------------------------------------------------------ GPU workload
+class Workload:
+    """One cache with a loaded prefix, the step's inputs in HBM, and its CUDA graphs."""
+
+    def __init__(self, cfg, layout, total_steps, seed, device):
+        import torch
+        from self_speculative_decode_b200.ripe import RipeCache
+        from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
+
+        self.cfg, self.layout, self.device = cfg, layout, device
+        N, L, Hq, kvH, d, R, T, B = (cfg[k] for k in ("N", "L", "Hq", "kvH", "d", "R", "T", "B"))
+        self.max_T = T + B * (total_steps + 4)
+        W = {"ripe": cfg["W"], "full": self.max_T, "deepest": 0}[layout]
+        self.W = W
+        self.cache = RipeCache(N, L, Hq, kvH, d, R, W, self.max_T, B)
+        for layer in range(L):
+            src = PlaneSource(N, kvH, d, R, T, cfg["rho"], seed, layer=layer, backend="torch", device=device)
+            for pl in range(R):
+                self.cache.load_prefix(layer, pl, [T] * N, src.plane(pl, "K"), src.plane(pl, "V"))
+            src.release()
+        bf = torch.bfloat16
+        self.q = torch.empty((L, R, N, B, Hq, d), dtype=bf, device=device)
+        self.k = torch.empty((L, R, N, B, kvH, d), dtype=bf, device=device)
+        self.v = torch.empty_like(self.k)
+        self.out = torch.empty_like(self.q)
+        for layer in range(L):
+            src = PlaneSource(N, kvH, d, R, T, cfg["rho"], seed, layer=layer, backend="torch", device=device)
+            for r in range(R):
+                self.k[layer, r] = src.block(0, r, B, "K")
+                self.v[layer, r] = src.block(0, r, B, "V")
+                self.q[layer, r] = src.queries(r, B, Hq)
+        draws = acceptance_draws(seed, total_steps + 2, N, B)
+        self.acc_host = draws
+        self.acc_table = torch.tensor(draws, dtype=torch.int32, device=device)
+        self.acc = torch.zeros(N, dtype=torch.int32, device=device)
+        torch.cuda.synchronize()
+        self.T0 = T
+
+    def _appends_and_verifies(self, verify_only=False):
+        c, cfg = self.cache, self.cfg
+        for r in range(cfg["R"]):
+            for layer in range(cfg["L"]):
+                if not verify_only:
+                    c.append_block(layer, r, self.k[layer, r], self.v[layer, r])
+                c.verify_attn(layer, r, self.q[layer, r], out=self.out[layer, r])
+
+    def capture(self):
+        import torch
+        c = self.cache
+        # put the block in place so the verify-only graph can be captured, then both graphs
+        for r in range(self.cfg["R"]):
+            for layer in range(self.cfg["L"]):
+                c.append_block(layer, r, self.k[layer, r], self.v[layer, r])
+        torch.cuda.synchronize()
+        n0 = c.launch_count()
+        self.g_verify = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_verify):
+            self._appends_and_verifies(verify_only=True)
+        self.launches_verify = c.launch_count() - n0
+        n0 = c.launch_count()
+        self.g_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_step):
+            self._appends_and_verifies()
+            c.commit_device(self.acc)
+        self.launches_step = c.launch_count() - n0
+        torch.cuda.synchronize()
+
+    def run_steps(self, first, count):
+        for i in range(first, first + count):
+            self.acc.copy_(self.acc_table[i], non_blocking=True)
+            self.g_step.replay()
+
+    def close(self):
+        assert self.cache.device_error() == 0, "device error word set"
+        self.cache.close()
+
+
+def time_region(fn, sync_group):
+    import torch
+    torch.cuda.synchronize()
+    if sync_group:
+        import torch.distributed as dist
+        dist.barrier()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record()
+    fn()
+    e.record()
+    torch.cuda.synchronize()
+    if sync_group:
+        import torch.distributed as dist
+        dist.barrier()
+    return s.elapsed_time(e)  # ms
+
+
+def max_over_ranks(x, dist_on):
+    if not dist_on:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def step_bytes(cfg, T_start, acc_rows):
+    """Verify bytes of every step, from the committed lengths each step starts with."""
+    T = list(T_start)
+    out = []
+    for row in acc_rows:
+        out.append(sum(verify_bytes(cfg, T, r) for r in range(cfg["R"])) * cfg["L"])
+        T = [t + int(a) for t, a in zip(T, row)]
+    return out, T
+
+
+def bench_layout(cfg, layout, args, seed, device, dist_on, want_extras):
+    import torch
+    wl = Workload(cfg, layout, args.warmup + 2 * args.steps + 2, seed, device)
+    wl.capture()
+    N = cfg["N"]
+    wl.run_steps(0, args.warmup)
+    T_start = wl.cache.sync_lengths()
+    res = {}
+    clocks = ClockSampler(gpu_id(torch.cuda.current_device())) if want_extras else None
+    if clocks:
+        clocks.start()
+    ms = time_region(lambda: wl.run_steps(args.warmup, args.steps), dist_on)
+    if clocks:
+        res["clocks"] = clocks.stop()
+    ms = max_over_ranks(ms, dist_on)
+    rows = wl.acc_host[args.warmup:args.warmup + args.steps]
+    per_step, T_end = step_bytes(cfg, T_start, rows)
+    T_check = wl.cache.sync_lengths()
+    assert T_check == T_end, (T_check, T_end)
+    nbytes = sum(per_step)
+    res.update(ms_per_step=ms / args.steps, bytes_per_step=nbytes / args.steps,
+               gbs=nbytes / (ms * 1e-3) / 1e9,
+               verified_tokens_per_s=N * cfg["B"] * args.steps / (ms * 1e-3),
+               accepted_tokens_per_s=float(rows.sum()) / (ms * 1e-3),
+               T_range=[min(T_start), max(T_end)], launches_per_step=wl.launches_step)
+    if want_extras:
+        # dominant kernel: verify, the same R*L launches as in the step, back to back (graph)
+        calls = cfg["R"] * cfg["L"]
+        reps = max(3, args.steps)
+        T_now = wl.cache.sync_lengths()
+        # a real block at the current lengths for the verify-only launches below
+        for r in range(cfg["R"]):
+            for layer in range(cfg["L"]):
+                wl.cache.append_block(layer, r, wl.k[layer, r], wl.v[layer, r])
+        vbytes = sum(verify_bytes(cfg, T_now, r) for r in range(cfg["R"])) * cfg["L"] / calls
+        vms = time_region(lambda: [wl.g_verify.replay() for _ in range(reps)], dist_on)
+        res["verify_warm"] = dict(us_per_launch=vms * 1e3 / (reps * calls), bytes_per_launch=vbytes)
+        # cold: L2 flushed (a 512 MB write) before every launch, each launch bracketed by events
+        flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        evs = []
+        for i in range(min(calls, 64)):
+            r, layer = divmod(i, cfg["L"])
+            flush.fill_(float(i))
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            wl.cache.verify_attn(layer, r % cfg["R"], wl.q[layer, r % cfg["R"]], out=wl.out[layer, r % cfg["R"]])
+            b.record()
+            evs.append((a, b, verify_bytes(cfg, T_now, r % cfg["R"])))
+        torch.cuda.synchronize()
+        tot_ms = sum(a.elapsed_time(b) for a, b, _ in evs)
+        res["verify_cold"] = dict(us_per_launch=tot_ms * 1e3 / len(evs),
+                                  bytes_per_launch=sum(x for _, _, x in evs) / len(evs))
+        del flush
+        res["e2e"] = e2e_steps(wl, args, dist_on)
+    wl.close()
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def e2e_steps(wl, args, dist_on):
+    """The same steps through the public API with host buffers: pinned host -> device copies of
+    the step's queries and block planes, the step, and the outputs copied back, all timed."""
+    import torch
+    hq = torch.empty(wl.q.shape, dtype=wl.q.dtype, pin_memory=True)
+    hk = torch.empty(wl.k.shape, dtype=wl.k.dtype, pin_memory=True)
+    hv = torch.empty(wl.v.shape, dtype=wl.v.dtype, pin_memory=True)
+    ho = torch.empty(wl.out.shape, dtype=wl.out.dtype, pin_memory=True)
+    hq.copy_(wl.q)
+    hk.copy_(wl.k)
+    hv.copy_(wl.v)
+    ha = torch.tensor(wl.acc_host, dtype=torch.int32).pin_memory()
+    first = args.warmup + args.steps
+    T_start = wl.cache.sync_lengths()
+
+    def run():
+        for i in range(first, first + args.steps):
+            wl.q.copy_(hq, non_blocking=True)
+            wl.k.copy_(hk, non_blocking=True)
+            wl.v.copy_(hv, non_blocking=True)
+            wl.acc.copy_(ha[i], non_blocking=True)
+            wl.g_step.replay()
+            ho.copy_(wl.out, non_blocking=True)
+
+    ms = max_over_ranks(time_region(run, dist_on), dist_on)
+    per_step, _ = step_bytes(wl.cfg, T_start, wl.acc_host[first:first + args.steps])
+    h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2 + wl.cfg["N"] * 4
+    return dict(value=sum(per_step) / (ms * 1e-3) / 1e9, unit="GB/s", ms_per_step=ms / args.steps,
+                h2d_bytes_per_step=h2d, d2h_bytes_per_step=ho.numel() * 2)
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(cfg, seconds, seed=0, loops=4):
+    """Time the CPU oracle on verify calls of layer 0 (loops 0..loops-1 and the deepest),
+    repeating until `seconds` of oracle time; returns (GB/s, calls, seconds, threads)."""
+    import numpy as np
+    from oracle import ripe_oracle as orc
+    from self_speculative_decode_b200.synth import PlaneSource
+
+    N, kvH, d, R, T, B, W = (cfg[k] for k in ("N", "kvH", "d", "R", "T", "B", "W"))
+    g = cfg["Hq"] // kvH
+    src = PlaneSource(N, kvH, d, R, T + B, cfg["rho"], seed)
+    oc = orc.OracleCache(N, 1, kvH, d, R, W, T + B, value_planes=set(range(loops)) | {R - 1})
+    for pl in range(R):
+        keep = pl < loops or pl == R - 1
+        k = src.plane(pl, "K") if keep else None
+        v = src.plane(pl, "V") if keep else None
+        oc.load_prefix(0, pl, [T] * N, k, v)
+    for pl in range(R):
+        keep = pl < loops or pl == R - 1
+        if keep:
+            kp, vp = src.plane(pl, "K"), src.plane(pl, "V")
+            kb = np.ascontiguousarray(kp[:, :, T:T + B].transpose(0, 2, 1, 3))
+            vb = np.ascontiguousarray(vp[:, :, T:T + B].transpose(0, 2, 1, 3))
+            oc.append(0, pl, kb, vb)
+        else:
+            oc.append(0, pl, None, None, B=B)
+    inputs = [(r, oc.verify_inputs(0, r)[:4], src.queries(r, B, cfg["Hq"])) for r in list(range(loops)) + [R - 1]]
+    spent, calls, nbytes = 0.0, 0, 0
+    while spent < seconds:
+        r, (Kr, Vr, Kl, Vl), q = inputs[calls % len(inputs)]
+        qf = orc.bf16_to_f64(q)
+        t0 = time.perf_counter()
+        orc.verify(oc.T, B, r, R, W, g, Kr, Vr, Kl, Vl, qf)
+        spent += time.perf_counter() - t0
+        calls += 1
+        nbytes += verify_bytes(cfg, [T] * N, r)
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return nbytes / spent / 1e9, calls, spent, threads
+
+
+def run_reference(args, cfg, rank):
+    """The oracle as the reference arm: each step is one bounded sample of the workload."""
+    if rank != 0:
+        return
+    per_step = []
+    calls_total = 0
+    for i in range(args.warmup + args.steps):
+        gbs, calls, sec, threads = oracle_sample(cfg, 0.5, seed=i)
+        if i >= args.warmup:
+            per_step.append((gbs, sec, calls))
+            calls_total += calls
+    value = sum(g * s for g, s, _ in per_step) / sum(s for _, s, _ in per_step)
+    ms = sum(s for _, s, _ in per_step) / len(per_step) * 1e3
+    sample = (f"{calls_total} oracle verify calls of layer 0 (loops 0-3 and {cfg['R'] - 1}), "
+              f"about 0.5 s of oracle time per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg["workload"], "layout": "ripe", "parallelism": "cpu oracle, OpenMP"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ripe", choices=["ripe", "reference"])
+    ap.add_argument("--config", default="huginn", choices=sorted(CONFIGS))
+    ap.add_argument("--layouts", default="ripe,full,deepest")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--seed", type=int, default=0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    from self_speculative_decode_b200 import ripe
+    ripe.lib()
+
+    layouts = [x for x in args.layouts.split(",") if x]
+    results = {}
+    for lay in layouts:
+        results[lay] = bench_layout(cfg, lay, args, args.seed + 1000 * rank, device, dist_on,
+                                    want_extras=(lay == layouts[0]))
+    main_l = layouts[0]
+    m = results[main_l]
+    peak, peak_kind = hbm_peak()
+    warm = m["verify_warm"]
+    cold = m["verify_cold"]
+    achieved = warm["bytes_per_launch"] / (warm["us_per_launch"] * 1e-6) / 1e9
+    achieved_cold = cold["bytes_per_launch"] / (cold["us_per_launch"] * 1e-6) / 1e9
+    value = m["gbs"] * world
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg["workload"], "layout": main_l,
+                   "step": "R*L x (append plane r + verify at loop r) + commit/evict, CUDA graph",
+                   "T_range": m["T_range"], "l2": "inputs larger than L2 (every step reads the whole cache)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": 100.0 * m["gbs"] / peak,
+        "verified_tokens_per_s": m["verified_tokens_per_s"] * world,
+        "accepted_tokens_per_s": m["accepted_tokens_per_s"] * world,
+        "layouts": {k: {x: v[x] for x in ("ms_per_step", "gbs", "verified_tokens_per_s", "bytes_per_step")}
+                    for k, v in results.items()},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "kernel": "ripe_verify_kernel", "launch_us": warm["us_per_launch"],
+                     "note": "R*L verify launches back to back as in the step (L2 warm)"},
+        "roofline_cold": {"achieved": achieved_cold, "frac": achieved_cold / peak,
+                          "launch_us": cold["us_per_launch"], "note": "L2 flushed before each launch"},
+        "e2e": m["e2e"],
+        "gpu_launches": m["launches_per_step"] * args.steps,
+        "clocks": m.get("clocks"),
+    }
+    if "full" in results and main_l == "ripe":
+        line["full_over_ripe_latency"] = results["full"]["ms_per_step"] / m["ms_per_step"]
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        gbs, calls, sec, threads = oracle_sample(cfg, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{calls} oracle verify calls of layer 0 (loops 0-3 and "
+                                          f"{cfg['R'] - 1}), {sec:.1f} s of oracle time"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist_on:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

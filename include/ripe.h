@@ -1,0 +1,199 @@
+/*
+ * ripe.h -- C ABI of the RIPE verify-attention library (libripe.so, sm_100a).
+ *
+ * A looped language model runs one block of layers R times per token, so each
+ * recurrent layer has R planes of keys and values per position; the verify
+ * pass of self-speculative decoding reads them at every loop r.  RIPE keeps
+ * the deepest plane (r = R-1) of every position and all R planes only for a
+ * window of the W most recent positions.
+ *   Source: "Prefix Keys and Values Matter Late: RIPE Caching for
+ *   Self-Speculative Decoding in Looped Language Models" (arXiv 2610.34436),
+ *   abstract, first, fourth and fifth sentences.
+ * Accept / rollback of a draft block follows the draft-then-verify scheme as
+ * described in the WaveFront Decoding write-up (rit.work blog, section "the
+ * draft and the check pass through the model at once"): the verified prefix of
+ * the block is kept, the full-depth token replaces the first mismatch, and the
+ * drafts after it are discarded.
+ *
+ * Conventions for every call:
+ *   - Device pointers are plain CUDA device addresses owned by the caller and
+ *     must stay valid until the work enqueued on `stream` has finished.
+ *     Host pointers are read before the call returns.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All device
+ *     work is enqueued on it; calls return after enqueueing.
+ *   - bf16 tensors are IEEE bfloat16, contiguous, row-major in the order given.
+ *   - Argument and state errors are detected on the host before anything is
+ *     enqueued and leave the cache unchanged.  A failed launch returns
+ *     RIPE_ECUDA.  Faults detected by a kernel (a wait that gave up, a block
+ *     that would overflow the capacity) set bits in a device error word read
+ *     by ripe_get_device_error(); kernels never trap.
+ *   - A cache handle is not thread-safe and must be used from one stream at a
+ *     time: calls on one handle share scratch memory on the device.
+ */
+#ifndef RIPE_H
+#define RIPE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct ripe_cache ripe_cache_t;
+
+/* Status codes returned by every call. */
+enum ripe_status {
+    RIPE_OK = 0,
+    RIPE_EINVAL = -1,    /* bad argument (shape, index, null pointer, unsupported size) */
+    RIPE_ENOMEM = -2,    /* device or host allocation failed */
+    RIPE_ECAPACITY = -3, /* committed + block positions would exceed max_T */
+    RIPE_ESTATE = -4,    /* call out of order (e.g. verify before the plane was appended) */
+    RIPE_ECUDA = -5      /* a CUDA runtime call or kernel launch failed */
+};
+
+/* How the window of full-depth positions is measured for a query at position p = T + j.
+ * QUERY_RELATIVE (default): key t reads plane r when t >= p - W; this is the rule under
+ *   which a window at least as long as the draft block makes batched verification
+ *   independent of how positions are split into blocks (RIPE abstract, fifth sentence).
+ * CACHE_RELATIVE: key t reads plane r when t >= T - W for every query of the block.
+ * In both modes the draft block's own keys read plane r (their deeper planes do not exist
+ * yet) and every other key reads the deepest plane R-1. */
+enum ripe_window_mode { RIPE_WINDOW_QUERY_RELATIVE = 0, RIPE_WINDOW_CACHE_RELATIVE = 1 };
+
+/* Device error bits reported by ripe_get_device_error(). */
+enum ripe_device_error {
+    RIPE_DEVERR_WAIT_TIMEOUT = 1u, /* a kernel gave up waiting for its own copies */
+    RIPE_DEVERR_CAPACITY = 2u,     /* a kernel saw T + B > max_T and skipped its work */
+    RIPE_DEVERR_ACCEPT = 4u        /* a device-side accepted length was outside [0, B] */
+};
+
+typedef struct ripe_stats {
+    int64_t stored_position_planes; /* sum over sequences of (position, plane) pairs kept for
+                                       the committed positions, per layer and key/value head:
+                                       T_n + min(W, T_n) * (R - 1) per sequence */
+    int64_t full_position_planes;   /* the same for the full cache: R * T_n per sequence */
+    int64_t kv_bytes;               /* device bytes of the key/value regions (all layers) */
+    int64_t scratch_bytes;          /* device bytes of per-call scratch and metadata */
+    int32_t deep_rows;              /* rows per (layer, sequence, kv head) of the deepest-plane region */
+    int32_t ring_slots;             /* slots per (layer, sequence, plane, kv head) of the window ring */
+    int32_t block_len;              /* B of the draft block in flight, 0 when none */
+    int32_t lengths_synced;         /* 1 when the host copy of T_n is current */
+} ripe_stats;
+
+/*
+ * Allocate a cache for `batch` sequences.
+ *   layers      recurrent layers L (>= 1)
+ *   q_heads     query heads Hq; kv_heads divides it, query head h uses kv head h / (Hq / kv_heads)
+ *   head_dim    d, one of 64, 96, 128
+ *   loops       R (1 .. 256); plane R-1 is the deepest
+ *   window      W >= 0; W >= max_T stores every plane (full cache), W = 0 keeps only the deepest
+ *   max_T       capacity per sequence: committed positions + draft block <= max_T
+ *   max_B       largest draft block (1 .. 64, and max_B * Hq / kv_heads <= 64)
+ *   window_mode enum ripe_window_mode
+ * Device layout (bf16):
+ *   deepest plane  K,V [L][batch][kv_heads][max(0, max_T - W)][d]   position t at row t
+ *   window ring    K,V [L][batch][R][kv_heads][S][d], S = min(W + max_B, max_T),
+ *                  position t at slot t mod S
+ * The library owns all cache memory and frees it in ripe_cache_free().  Every cache starts
+ * empty (T_n = 0).  On failure *out is NULL.
+ */
+int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_dim, int loops,
+                     int window, int max_T, int max_B, int window_mode, ripe_cache_t **out);
+
+/* Free a cache and its device memory (synchronises the device first).  NULL is a no-op. */
+int ripe_cache_free(ripe_cache_t *c);
+
+/*
+ * Load one plane of a prefix for one layer (RIPE abstract, fourth sentence: the deepest
+ * plane is kept everywhere, the other planes only inside the window).
+ *   T       host int32[batch], committed prefix length of each sequence; the first load
+ *           sets the lengths, later loads (other layers or planes) must pass the same values
+ *   plane   0 .. R-1
+ *   k, v    device bf16 [batch][kv_heads][ld_t][d], positions 0 .. T_n - 1 of this plane
+ *   ld_t    row stride in positions, >= max over n of T_n
+ * Plane R-1 is stored for every position; other planes only for positions t >= T_n - W.
+ * Requires no draft block in flight (RIPE_ESTATE) and T_n + 1 <= max_T (RIPE_ECAPACITY).
+ */
+int ripe_load_prefix(ripe_cache_t *c, int layer, int plane, const int32_t *T, const void *k,
+                     const void *v, int64_t ld_t, void *stream);
+
+/*
+ * Append plane r of the current draft block of one layer: block position j of sequence n
+ * (absolute position T_n + j) goes to ring slot (T_n + j) mod S of plane r.
+ *   B      block length, 1 .. max_B; all appends of one block use the same B
+ *   k, v   device bf16 [batch][B][kv_heads][d]
+ * The block's planes are computed while it is verified (RIPE abstract, first sentence:
+ * verification runs all R loops), so plane r must be appended before ripe_verify_attn(.., r).
+ * Errors: RIPE_ECAPACITY if T_n + B > max_T for some n.
+ */
+int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, const void *v,
+                      void *stream);
+
+/*
+ * Verification attention of the draft block at loop r for one layer.
+ * For query head h of block position j of sequence n (p = T_n + j) and every key t <= p:
+ * the key/value plane is r when t >= T_n (draft block) or t is inside the window (see
+ * enum ripe_window_mode), else the deepest plane R-1; out is the causal softmax attention
+ * softmax_t(scale * <q, K_plane[t]>) . V_plane[t].
+ *   q      device bf16 [batch][B][q_heads][d]
+ *   out    device bf16 [batch][B][q_heads][d], rounded to nearest even from fp32
+ *   lse    device fp32 [batch][B][q_heads] natural-log softmax normaliser, or NULL
+ *   scale  logit scale (1/sqrt(d) for unscaled queries)
+ * Requires plane r of the block appended for this layer (else RIPE_ESTATE).
+ * Work: split-KV over the deepest-plane region and the window ring in one persistent
+ * launch; partial results are merged in the same launch through per-call scratch owned by
+ * the cache.
+ */
+int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out, float *lse,
+                     float scale, void *stream);
+
+/*
+ * Accept a prefix of the draft block of every sequence and roll back the rest
+ * (WaveFront write-up, draft-then-verify): accepted_len[n] in 0 .. B positions of the block
+ * become committed, T_n += accepted_len[n]; the other block positions are discarded.
+ * Positions that leave the window (t < T_n - W) move their deepest plane from the ring into
+ * the deepest-plane region, and planes 0 .. R-2 of them are dropped (RIPE abstract, fourth
+ * sentence).  Requires every plane of the block appended for every layer (RIPE_ESTATE).
+ *   accepted_len  host int32[batch]
+ */
+int ripe_commit(ripe_cache_t *c, const int32_t *accepted_len, void *stream);
+
+/*
+ * Same as ripe_commit with the accepted lengths in device memory (device int32[batch]), for
+ * decoders that compute acceptance on the GPU.  Values outside 0 .. B are clamped and set
+ * RIPE_DEVERR_ACCEPT.  The host copy of T_n becomes stale until ripe_sync_lengths(); until
+ * then host-side capacity checks assume every device commit accepted the whole block.
+ */
+int ripe_commit_device(ripe_cache_t *c, const int32_t *accepted_len, void *stream);
+
+/* Copy T_n from the device to the host copy (synchronises `stream`); optional T_out[batch]. */
+int ripe_sync_lengths(ripe_cache_t *c, int32_t *T_out, void *stream);
+
+/* Counters and geometry of the cache (host copy of the state; no device work). */
+int ripe_cache_stats(const ripe_cache_t *c, ripe_stats *st);
+
+/*
+ * Logical view of one sequence of one layer, for tests: every position t < Tv = T_n + B
+ * (B = block in flight, or 0) and every plane.
+ *   k_out, v_out    device bf16 [R][kv_heads][Tv][d]; absent (position, plane) pairs are zero
+ *   plane_present   device uint8 [R][Tv]; 1 where the cache stores that plane of that position
+ * Requires synced lengths (RIPE_ESTATE otherwise).
+ */
+int ripe_cache_export(ripe_cache_t *c, int n, int layer, void *k_out, void *v_out,
+                      uint8_t *plane_present, void *stream);
+
+/* Read and clear the device error word (synchronises `stream`); *err_out gets its bits. */
+int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream);
+
+/* Number of kernel launches the library has enqueued since the cache was allocated. */
+int64_t ripe_launch_count(const ripe_cache_t *c);
+
+/* Static description of a status code. */
+const char *ripe_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RIPE_H */

@@ -154,9 +154,11 @@ class OracleCache:
       * commit(a): block positions j < a_n become committed, the rest are
         discarded; then positions that left the window drop planes 0 .. R-2.
     ``W >= max_T`` is the full cache, ``W = 0`` keeps only the deepest plane.
+    ``value_planes`` (optional) limits which planes keep their bf16 values, to save host
+    memory on large shapes; presence is tracked for every plane either way.
     """
 
-    def __init__(self, N, L, kvH, d, R, W, max_T, mode=QUERY_RELATIVE):
+    def __init__(self, N, L, kvH, d, R, W, max_T, mode=QUERY_RELATIVE, value_planes=None):
         self.N, self.L, self.kvH, self.d, self.R, self.W = N, L, kvH, d, R, W
         self.max_T, self.mode = max_T, mode
         self.T = np.zeros(N, dtype=np.int64)
@@ -166,6 +168,10 @@ class OracleCache:
         self._K = {}
         self._V = {}
         self._prefix_set = False
+        self.value_planes = None if value_planes is None else set(int(p) for p in value_planes)
+
+    def _keeps(self, plane):
+        return self.value_planes is None or plane in self.value_planes
 
     def _arr(self, store, layer, plane):
         key = (layer, plane)
@@ -188,27 +194,32 @@ class OracleCache:
             raise ValueError("prefix lengths differ between calls")
         self.T = T.copy()
         self._prefix_set = True
-        K, V = self._arr(self._K, layer, plane), self._arr(self._V, layer, plane)
+        keep = self._keeps(plane)
         for n in range(self.N):
             lo = 0 if plane == self.R - 1 else max(0, int(T[n]) - self.W)
             hi = int(T[n])
-            K[n, :, lo:hi] = k[n, :, lo:hi]
-            V[n, :, lo:hi] = v[n, :, lo:hi]
+            if keep:
+                self._arr(self._K, layer, plane)[n, :, lo:hi] = k[n, :, lo:hi]
+                self._arr(self._V, layer, plane)[n, :, lo:hi] = v[n, :, lo:hi]
             self.present[layer, plane, n, lo:hi] = True
 
-    def append(self, layer, r, k, v):
-        """Plane r of the draft block for one layer: k, v bits [N][B][kvH][d]."""
-        B = k.shape[1]
+    def append(self, layer, r, k, v, B=None):
+        """Plane r of the draft block for one layer: k, v bits [N][B][kvH][d].
+
+        For a plane outside ``value_planes`` k and v may be None (then B is required).
+        """
+        B = k.shape[1] if k is not None else int(B)
         if self.B and B != self.B:
             raise ValueError("block length changed inside a block")
         if np.any(self.T + B > self.max_T):
             raise ValueError("capacity")
         self.B = B
-        K, V = self._arr(self._K, layer, r), self._arr(self._V, layer, r)
+        keep = self._keeps(r)
         for n in range(self.N):
             t0 = int(self.T[n])
-            K[n, :, t0:t0 + B] = np.transpose(k[n], (1, 0, 2))
-            V[n, :, t0:t0 + B] = np.transpose(v[n], (1, 0, 2))
+            if keep:
+                self._arr(self._K, layer, r)[n, :, t0:t0 + B] = np.transpose(k[n], (1, 0, 2))
+                self._arr(self._V, layer, r)[n, :, t0:t0 + B] = np.transpose(v[n], (1, 0, 2))
             self.present[layer, r, n, t0:t0 + B] = True
         self.appended[layer, r] = True
 
@@ -256,6 +267,8 @@ class OracleCache:
         """Verification attention of the current block at loop r: (out, lse) in fp64."""
         if not self.appended[layer, r]:
             raise RuntimeError("verify before plane r of the block was appended")
+        if not (self._keeps(r) and self._keeps(self.R - 1)):
+            raise RuntimeError("verify needs the values of planes r and R-1")
         Kr, Vr, Kl, Vl, _ = self.verify_inputs(layer, r)
         return verify(self.T, self.B, r, self.R, self.W, g, Kr, Vr, Kl, Vl,
                       bf16_to_f64(q_bits), scale, self.mode)

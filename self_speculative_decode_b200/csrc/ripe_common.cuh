@@ -1,0 +1,240 @@
+// Internal definitions shared by the RIPE library's translation units (sm_100a).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "ripe.h"
+
+namespace ripe {
+
+constexpr int kMaxBatch = 1024;   // sequences per cache (accepted lengths travel as kernel parameters)
+constexpr int kMaxLoops = 256;    // R
+constexpr int kTileRows = 64;     // keys per pipeline stage
+constexpr int kBoxCols = 32;      // bf16 per TMA box row: 64 bytes, 64-byte swizzle
+constexpr int kBoxBytes = kTileRows * 64;  // one box slot in shared memory (4 KB)
+constexpr int kStages = 4;        // TMA pipeline depth of the verify kernel
+constexpr int kMaxQueryRows = 64; // B * (Hq / kvH) per key/value head
+
+// Bounded waits: a kernel that does not see its copies land within this many polls
+// records RIPE_DEVERR_WAIT_TIMEOUT and stops (it never traps).
+constexpr uint32_t kWaitPolls = 1u << 26;
+
+struct HostIntArray {
+    int32_t v[kMaxBatch];
+};
+
+}  // namespace ripe
+
+// The opaque handle of the C ABI.
+struct ripe_cache {
+    // geometry
+    int N, L, Hq, kvH, g, d, R, W, max_T, max_B, mode;
+    int ring_slots;  // S = min(W + max_B, max_T)
+    int deep_rows;   // max(0, max_T - W)
+    int deep_box, ring_box;  // TMA box heights (<= 64)
+    int device, num_sms;
+    // device memory
+    __nv_bfloat16 *Kd, *Vd;  // [L][N][kvH][deep_rows][d]
+    __nv_bfloat16 *Kw, *Vw;  // [L][N][R][kvH][S][d]
+    int32_t *T_dev;          // [N]
+    uint32_t *err_dev;       // device error word
+    float *part_o;           // [part_slots][part_rows][d]
+    float *part_ml;          // [part_slots][part_rows][2]
+    int32_t *counters;       // [N * kvH] arrivals per (sequence, kv head), reset by the last arrival
+    int part_slots, part_rows;
+    CUtensorMap tm_Kd, tm_Vd, tm_Kw, tm_Vw;
+    // host copy of the state
+    std::vector<int32_t> T;   // committed lengths (an upper bound when !synced)
+    int B_cur;                // block in flight (0 = none)
+    std::vector<uint8_t> appended;  // [L][R] planes of the block appended
+    bool prefix_set, synced;
+    int64_t kv_bytes, scratch_bytes;
+    int64_t launches;
+};
+
+namespace ripe {
+
+// ---------------------------------------------------------------- tile plan
+// The keys of one (sequence, kv head) at loop r form a list of tiles:
+//   DEEP  the deepest-plane region, positions [0, D), D = max(0, T - W)
+//   RING  positions [D, T + B) at plane r from the window ring (window + draft block)
+//   DUAL  positions [D, min(T, T + B - 1 - W)) at plane R-1 from the ring: window keys
+//         that are older than W for the later queries of the block (query-relative rule)
+// Ring ranges are cut where the ring wraps, so every tile is one box of consecutive slots.
+enum TileKind { kDeep = 0, kRing = 1, kDual = 2 };
+
+struct PlanArgs {
+    int W, B, R, r, ring_slots, deep_box, ring_box, mode_eff;
+};
+
+struct SeqGeom {
+    int T, D, nd;
+    int ring_len, ring_first, nr1, nr;
+    int dual_len, dual_first, ndl1, ndl;
+    int total;
+};
+
+struct Tile {
+    int kind, t0, cnt, y, plane;
+};
+
+__host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+__host__ __device__ __forceinline__ SeqGeom seq_geom(int T, const PlanArgs &a) {
+    SeqGeom s;
+    s.T = T;
+    s.D = T - a.W > 0 ? T - a.W : 0;
+    s.nd = cdiv(s.D, a.deep_box);
+    const int s0 = s.D % a.ring_slots;
+    s.ring_len = T + a.B - s.D;
+    s.ring_first = s.ring_len < a.ring_slots - s0 ? s.ring_len : a.ring_slots - s0;
+    s.nr1 = cdiv(s.ring_first, a.ring_box);
+    s.nr = s.nr1 + cdiv(s.ring_len - s.ring_first, a.ring_box);
+    int dl = 0;
+    if (a.mode_eff == 0) {
+        const int hi = T < T + a.B - 1 - a.W ? T : T + a.B - 1 - a.W;
+        dl = hi - s.D > 0 ? hi - s.D : 0;
+    }
+    s.dual_len = dl;
+    s.dual_first = dl < a.ring_slots - s0 ? dl : a.ring_slots - s0;
+    s.ndl1 = cdiv(s.dual_first, a.ring_box);
+    s.ndl = s.ndl1 + cdiv(s.dual_len - s.dual_first, a.ring_box);
+    s.total = s.nd + s.nr + s.ndl;
+    return s;
+}
+
+__host__ __device__ __forceinline__ Tile tile_at(const SeqGeom &s, int lt, const PlanArgs &a) {
+    Tile t;
+    if (lt < s.nd) {
+        t.kind = kDeep;
+        t.t0 = lt * a.deep_box;
+        t.cnt = (s.D - t.t0) < a.deep_box ? (s.D - t.t0) : a.deep_box;
+        t.y = t.t0;
+        t.plane = a.R - 1;
+        return t;
+    }
+    lt -= s.nd;
+    int len, first, n1;
+    if (lt < s.nr) {
+        len = s.ring_len; first = s.ring_first; n1 = s.nr1;
+        t.kind = kRing; t.plane = a.r;
+    } else {
+        lt -= s.nr;
+        len = s.dual_len; first = s.dual_first; n1 = s.ndl1;
+        t.kind = kDual; t.plane = a.R - 1;
+    }
+    int off, seg_end;
+    if (lt < n1) { off = lt * a.ring_box; seg_end = first; }
+    else { off = first + (lt - n1) * a.ring_box; seg_end = len; }
+    t.t0 = s.D + off;
+    t.cnt = (seg_end - off) < a.ring_box ? (seg_end - off) : a.ring_box;
+    t.y = (s.D + off) % a.ring_slots;
+    return t;
+}
+
+// ---------------------------------------------------------------- PTX wrappers
+#if defined(__CUDACC__)
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete; false after kWaitPolls polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kWaitPolls; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 3-D tiled TMA load (no multicast) completing on an mbarrier.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, uint32_t bar, int x,
+                                            int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr)
+                 : "memory");
+}
+
+// D = A(16x16, bf16, row) * B(16x8, bf16, col) + D, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+#endif
+
+// ---------------------------------------------------------------- launchers (defined per .cu)
+int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
+                  float scale, cudaStream_t s);
+int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const void *v,
+                  cudaStream_t s);
+int launch_commit(ripe_cache *c, const int32_t *acc_host, const int32_t *acc_dev, cudaStream_t s);
+int launch_load_prefix(ripe_cache *c, int layer, int plane, const int32_t *T, const void *k,
+                       const void *v, int64_t ld_t, cudaStream_t s);
+int launch_export(ripe_cache *c, int n, int layer, void *k_out, void *v_out, uint8_t *present,
+                  cudaStream_t s);
+int verify_smem_bytes(int d, int wr, int N);
+int set_verify_attributes(int d, int N);
+
+}  // namespace ripe

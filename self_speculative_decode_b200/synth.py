@@ -71,6 +71,7 @@ class PlaneSource:
         if backend not in ("numpy", "torch"):
             raise ValueError("backend must be 'numpy' or 'torch'")
         self.shape = (N, kvH, length, d)
+        self._deep = {}
 
     # -- raw N(0,1) draws ------------------------------------------------------
     def _normal(self, parts, shape):
@@ -94,11 +95,17 @@ class PlaneSource:
         deep_id, noise_id = (K_DEEP, K_NOISE) if which == "K" else (V_DEEP, V_NOISE)
         if self.independent:
             return self._to_bf16(self._normal((noise_id, r), self.shape))
-        D = self._normal((deep_id,), self.shape)
+        if deep_id not in self._deep:
+            self._deep[deep_id] = self._normal((deep_id,), self.shape)
+        D = self._deep[deep_id]
         if r == self.R - 1:
             return self._to_bf16(D)
         eps = self._normal((noise_id, r), self.shape)
         return self._to_bf16(D + (self.rho ** r) * eps)
+
+    def release(self):
+        """Drop the cached deepest-plane draws."""
+        self._deep.clear()
 
     # -- draft blocks drawn per decoding step (streaming workloads) -------------
     def block(self, step: int, r: int, B: int, which: str = "K"):
