@@ -122,7 +122,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     const long long s_slots = static_cast<long long>(c->W) + max_B;
     c->ring_slots = static_cast<int>(s_slots < max_T ? s_slots : max_T);
     c->deep_rows = max_T - c->W;
-    c->deep_box = c->deep_rows < kTileRows ? (c->deep_rows > 0 ? c->deep_rows : 1) : kTileRows;
+    c->deep_box = (c->deep_rows == 0 || c->deep_rows >= kTileRows) ? kTileRows : c->deep_rows;
     c->ring_box = c->ring_slots < kTileRows ? c->ring_slots : kTileRows;
     c->T.assign(batch, 0);
     c->B_cur = 0;

@@ -20,9 +20,9 @@ constexpr int kBoxBytes = kTileRows * 64;  // one box slot in shared memory (4 K
 constexpr int kStages = 4;        // TMA pipeline depth of the verify kernel
 constexpr int kMaxQueryRows = 64; // B * (Hq / kvH) per key/value head
 
-// Bounded waits: a kernel that does not see its copies land within this many polls
-// records RIPE_DEVERR_WAIT_TIMEOUT and stops (it never traps).
-constexpr uint32_t kWaitPolls = 1u << 26;
+// Bounded waits: a kernel that does not see its copies land within this time records
+// RIPE_DEVERR_WAIT_TIMEOUT and stops (it never traps).
+constexpr unsigned long long kWaitNs = 4000000000ull;
 
 struct HostIntArray {
     int32_t v[kMaxBatch];
@@ -172,15 +172,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false after kWaitPolls polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
 }
 
-__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+// Wait for the phase with the given parity to complete; false after kWaitNs nanoseconds.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (;;) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > kWaitNs) return false;
+    }
 }
 
 // 3-D tiled TMA load (no multicast) completing on an mbarrier.
@@ -219,10 +225,40 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Transpose of an 8x8 bf16 matrix held one row-pair per lane (row lane/4, cols 2*(lane%4)+{0,1}).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t a) {
+    uint32_t d;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
+    return d;
+}
+
+// Programmatic dependent launch: wait for the previous kernel in the stream to finish (and its
+// memory to be visible) / allow the next kernel to be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 #endif
+
+// Launch with programmatic stream serialization: the kernel may start while the previous one
+// drains; every such kernel calls pdl_wait() before touching memory a previous kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
 
 // ---------------------------------------------------------------- launchers (defined per .cu)
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
@@ -234,7 +270,6 @@ int launch_load_prefix(ripe_cache *c, int layer, int plane, const int32_t *T, co
                        const void *v, int64_t ld_t, cudaStream_t s);
 int launch_export(ripe_cache *c, int n, int layer, void *k_out, void *v_out, uint8_t *present,
                   cudaStream_t s);
-int verify_smem_bytes(int d, int wr, int N);
 int set_verify_attributes(int d, int N);
 
 }  // namespace ripe

@@ -28,6 +28,8 @@ __global__ void ripe_append_kernel(uint4 *__restrict__ Kw, uint4 *__restrict__ V
                                    const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                    const int32_t *__restrict__ T, uint32_t *err, int N, int B, int kvH,
                                    int d8, int R, int S, int layer, int r, int max_T) {
+    pdl_wait();
+    pdl_trigger();
     const size_t total = static_cast<size_t>(N) * B * kvH * d8;
     for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
          idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
@@ -55,10 +57,10 @@ int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const v
     int blocks = static_cast<int>((total + 255) / 256);
     if (blocks > 4 * c->num_sms) blocks = 4 * c->num_sms;
     if (blocks < 1) blocks = 1;
-    ripe_append_kernel<<<blocks, 256, 0, s>>>(reinterpret_cast<uint4 *>(c->Kw), reinterpret_cast<uint4 *>(c->Vw),
-                                              static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
-                                              c->T_dev, c->err_dev, c->N, B, c->kvH, d8, c->R, c->ring_slots,
-                                              layer, r, c->max_T);
+    launch_pdl(ripe_append_kernel, dim3(blocks), dim3(256), 0, s, reinterpret_cast<uint4 *>(c->Kw),
+               reinterpret_cast<uint4 *>(c->Vw), static_cast<const uint4 *>(k), static_cast<const uint4 *>(v),
+               static_cast<const int32_t *>(c->T_dev), c->err_dev, c->N, B, c->kvH, d8, c->R, c->ring_slots, layer,
+               r, c->max_T);
     c->launches += 1;
     return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
@@ -83,6 +85,8 @@ __global__ void ripe_evict_kernel(uint4 *__restrict__ Kd, uint4 *__restrict__ Vd
                                   const int32_t *__restrict__ T, const HostIntArray acc_h,
                                   const int32_t *acc_d, uint32_t *err, int N, int B, int kvH, int d8,
                                   int R, int S, int W, int deep_rows) {
+    pdl_wait();
+    pdl_trigger();
     const int layer = blockIdx.x / N;
     const int n = blockIdx.x - layer * N;
     const int Tn = T[n];
@@ -106,6 +110,8 @@ __global__ void ripe_evict_kernel(uint4 *__restrict__ Kd, uint4 *__restrict__ Vd
 
 __global__ void ripe_commit_lengths_kernel(int32_t *T, const HostIntArray acc_h, const int32_t *acc_d,
                                            uint32_t *err, int N, int B) {
+    pdl_wait();
+    pdl_trigger();
     for (int n = threadIdx.x; n < N; n += blockDim.x) T[n] += accepted(acc_h, acc_d, n, B, err, true);
 }
 
@@ -118,15 +124,15 @@ int launch_commit(ripe_cache *c, const int32_t *acc_host, const int32_t *acc_dev
         int gy = (work + 255) / 256;
         if (gy < 1) gy = 1;
         dim3 grid(c->L * c->N, gy);
-        ripe_evict_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<uint4 *>(c->Kd), reinterpret_cast<uint4 *>(c->Vd),
-                                               reinterpret_cast<const uint4 *>(c->Kw),
-                                               reinterpret_cast<const uint4 *>(c->Vw), c->T_dev, ah, acc_dev,
-                                               c->err_dev, c->N, c->B_cur, c->kvH, d8, c->R, c->ring_slots,
-                                               c->W, c->deep_rows);
+        launch_pdl(ripe_evict_kernel, grid, dim3(256), 0, s, reinterpret_cast<uint4 *>(c->Kd),
+                   reinterpret_cast<uint4 *>(c->Vd), reinterpret_cast<const uint4 *>(c->Kw),
+                   reinterpret_cast<const uint4 *>(c->Vw), static_cast<const int32_t *>(c->T_dev), ah, acc_dev,
+                   c->err_dev, c->N, c->B_cur, c->kvH, d8, c->R, c->ring_slots, c->W, c->deep_rows);
         c->launches += 1;
         if (cudaGetLastError() != cudaSuccess) return RIPE_ECUDA;
     }
-    ripe_commit_lengths_kernel<<<1, 256, 0, s>>>(c->T_dev, ah, acc_dev, c->err_dev, c->N, c->B_cur);
+    launch_pdl(ripe_commit_lengths_kernel, dim3(1), dim3(256), 0, s, c->T_dev, ah, acc_dev, c->err_dev, c->N,
+               c->B_cur);
     c->launches += 1;
     return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }

@@ -12,17 +12,24 @@
 //     that later queries of the block see at the deepest plane (query-relative window).
 //     All lists are concatenated and cut into equal contiguous chunks, one per CTA, so
 //     ragged lengths and the three layouts (full, RIPE, deepest-only) balance the same way.
-//   * One producer warp streams 64-key K/V tiles with 3-D TMA loads (64-byte swizzle, no
-//     multicast) into a 4-stage shared-memory ring guarded by mbarriers.
-//   * Consumer warps: each owns 16 query rows (B positions x GQA group, so one K/V read
-//     serves the whole group) and 16 keys of each tile; S = Q K^T and O += P V run on the
-//     tensor cores (mma.sync m16n8k16 bf16 -> fp32); fp32 online softmax in base 2 with
-//     quad shuffles for the row max.
+//   * One producer thread streams 64-key K/V tiles with 3-D TMA loads (64-byte swizzle, no
+//     multicast) into a shared-memory ring of NS stages guarded by mbarriers, and writes a
+//     small descriptor of each tile (sequence, kv head, kind, first key, count) beside it.
+//   * Consumer warps work on the transposed problem S^T = K Q^T (keys on the MMA's M side,
+//     the B x group query rows on its N side, so an 8-row block is not padded to 16), with
+//     mma.sync m16n8k16 bf16 -> fp32.  P^T is moved into the B-operand layout of
+//     O^T += V^T P^T with movmatrix.  Every query row of one kv head is served by the same
+//     K/V tile (GQA group sharing).  Two groups of warps consume alternate tiles.
+//   * Online softmax in base 2; the reference maximum only moves when a tile's maximum
+//     exceeds it by more than 8 (so probabilities stay <= 2^8), which skips most O rescales
+//     and is exact.  Full deepest-plane tiles take a path without masks.
 //   * A CTA that covers a whole (sequence, kv head) writes the output directly.  Otherwise
 //     it writes an unnormalised partial (o, m, l); the last CTA to arrive (atomic counter,
 //     no spinning) merges the partials by log-sum-exp and writes out / lse.
 //   * Every wait is bounded: on timeout the kernel records RIPE_DEVERR_WAIT_TIMEOUT, drains
-//     its own copies in flight and returns without writing results.
+//     its own copies in flight and returns without writing further results.
+#include <type_traits>
+
 #include "ripe_common.cuh"
 
 namespace ripe {
@@ -37,70 +44,86 @@ struct VerifyArgs {
     int32_t *counters;
     uint32_t *err;
     PlanArgs plan;
-    int N, kvH, g, Hq, B, R, layer, Mq, part_rows;
+    int N, kvH, g, Hq, B, R, layer, Mq, min_chunk;
     float scale_log2;
 };
 
-template <int D, int WR>
+constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
+#ifndef RIPE_MIN_CHUNK
+#define RIPE_MIN_CHUNK 4                // at least this many 64-key tiles per CTA
+#endif
+constexpr float kLazyMax = 8.f;     // log2 headroom before the softmax reference moves
+
+// Query-side shapes: NQT 8-query tiles per warp, WR row groups, WK key groups per tile,
+// TG tile groups consuming alternate tiles.
+template <int D, int NQT, int WR, int WK, int TG>
 struct VCfg {
-    static constexpr int WK = (WR >= 4) ? 2 : 4;      // key groups per tile
-    static constexpr int NCW = WR * WK;               // consumer warps
-    static constexpr int THREADS = (NCW + 1) * 32;    // + one producer warp
-    static constexpr int NBOX = D / kBoxCols;         // TMA boxes per K (or V) tile
+    static constexpr int NQ = 8 * NQT;             // queries per warp
+    static constexpr int ROWS = NQ * WR;           // query rows per (sequence, kv head)
+    static constexpr int GW = WR * WK;             // warps per tile group
+    static constexpr int NCW = GW * TG;            // consumer warps
+    static constexpr int THREADS = (NCW + 1) * 32; // + the producer warp
+    static constexpr int SB = 4 / WK;              // 16-key sub-blocks per warp per tile
+    static constexpr int NBOX = D / kBoxCols;
     static constexpr int STAGE_BYTES = 2 * NBOX * kBoxBytes;
-    static constexpr int MERGE_FLOATS = NCW * 16 * D;
-    static constexpr int MLF = NCW * 16 * 2;
+    static constexpr int DP = D + 4;               // merge-buffer row stride (no bank conflicts)
+    static constexpr int MERGE_FLOATS = NCW * NQ * DP;
+    static constexpr int MLF = NCW * NQ * 2 + ROWS * (TG * WK + 2);
+    static constexpr int MISC = 1024 /*align*/ + 1024 /*bars, descriptors, flags*/;
+    static constexpr int AVAIL = kSmemLimit - MISC - 4 * (MERGE_FLOATS + MLF) - 4 * (2 * kMaxBatch + 2);
+    static constexpr int NS_RAW = AVAIL / STAGE_BYTES > 8 ? 8 : AVAIL / STAGE_BYTES;
+    static constexpr int NS = NS_RAW - NS_RAW % TG;
+    static_assert(NS >= 2, "not enough shared memory for the pipeline");
+    static constexpr int SMEM_FIXED = MISC + NS * STAGE_BYTES + 4 * (MERGE_FLOATS + MLF);
+    // the end-of-CTA merge keeps m and l of up to 256 partials per query row in the stage buffers
+    static_assert(NS * STAGE_BYTES >= 2 * 256 * ROWS * 4, "stage buffers too small for the merge");
 };
 
-__host__ __device__ constexpr int verify_smem_fixed(int D, int WR) {
-    return 1024 /* alignment slack */ + kStages * 2 * (D / kBoxCols) * kBoxBytes +
-           ((WR >= 4 ? 2 : 4) * WR) * 16 * (D + 2) * 4 + 2 * kStages * 8 + 16 * 4;
-}
-
-int verify_smem_bytes(int d, int wr, int N) {
-    return verify_smem_fixed(d, wr) + (2 * N + 2) * 4;
-}
-
-// Walks the concatenated tile lists in order.
-struct TileIter {
-    const int *cum;   // cum[n] = first global tile of sequence n
-    const int *Ts;    // T per sequence
-    int n, kh, lt;
-    SeqGeom s;
-
-    __device__ void start(int gt, int N, int kvH, const PlanArgs &a) {
-        n = 0;
-        while (n + 1 < N && cum[n + 1] <= gt) ++n;
-        s = seq_geom(Ts[n], a);
-        const int rel = gt - cum[n];
-        kh = rel / s.total;
-        lt = rel - kh * s.total;
-    }
-    __device__ void next(int N, int kvH, const PlanArgs &a) {
-        if (++lt < s.total) return;
-        lt = 0;
-        if (++kh < kvH) return;
-        kh = 0;
-        if (++n < N) s = seq_geom(Ts[n], a);
-    }
+struct TileDesc {
+    int pair, n, kh, T, kind, t0, cnt, pad;
 };
 
-template <int D, int WR>
-__global__ void __launch_bounds__(VCfg<D, WR>::THREADS, 1)
+template <class C>
+__host__ __device__ constexpr int smem_bytes_for(int N) {
+    return C::SMEM_FIXED + (2 * N + 2) * 4;
+}
+
+// index of the last sequence whose first tile is <= gt
+__device__ __forceinline__ int seq_of(const int *cum, int N, int gt) {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (cum[mid] <= gt) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ int pair_of(const int *cum, int N, int kvH, int gt) {
+    const int n = seq_of(cum, N, gt);
+    const int tot = (cum[n + 1] - cum[n]) / kvH;
+    return n * kvH + (gt - cum[n]) / tot;
+}
+
+template <int D, int NQT, int WR, int WK, int TG>
+__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS, 1)
 ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_constant__ CUtensorMap tmVd,
                    const __grid_constant__ CUtensorMap tmKw, const __grid_constant__ CUtensorMap tmVw,
                    const VerifyArgs a) {
-    using C = VCfg<D, WR>;
+    using C = VCfg<D, NQT, WR, WK, TG>;
+    constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *stages = base;
-    float *mo = reinterpret_cast<float *>(base + kStages * C::STAGE_BYTES);  // [NCW][16][D]
-    float *mml = mo + C::MERGE_FLOATS;                                       // [NCW][16][2]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);             // full, empty
-    int *sflag = reinterpret_cast<int *>(bars + 2 * kStages);                // [16]
-    int *cum = sflag + 16;                                                   // [N + 1]
-    int *Ts = cum + a.N + 1;                                                 // [N]
+    float *mo = reinterpret_cast<float *>(base + NS * C::STAGE_BYTES);   // [NCW][NQ][DP]
+    float *mml = mo + C::MERGE_FLOATS;                                   // [NCW][NQ][2]
+    float *wq = mml + C::NCW * C::NQ * 2;                                // [ROWS][TG*WK] weights
+    float *fin = wq + C::ROWS * TG * WK;                                 // [ROWS][2] final M, L
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);         // full[NS], empty[NS]
+    TileDesc *sdesc = reinterpret_cast<TileDesc *>(bars + 2 * NS);       // [NS]
+    int *sflag = reinterpret_cast<int *>(sdesc + NS);                    // [16]
+    int *cum = sflag + 16;                                               // [N + 1]
+    int *Ts = cum + a.N + 1;                                             // [N]
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -108,27 +131,28 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const PlanArgs &pa = a.plan;
     const int N = a.N, kvH = a.kvH;
 
-    // ---- per-sequence tile counts and their prefix sums
-    for (int n = tid; n < N; n += blockDim.x) {
-        const int T = a.T[n];
-        Ts[n] = T;
-        cum[n + 1] = seq_geom(T, pa).total * kvH;
-    }
     if (tid == 0) {
-        cum[0] = 0;
-        sflag[0] = 0;  // last-arrival flag
         sflag[1] = 0;  // abort flag
-        for (int s = 0; s < kStages; ++s) {
+        sflag[3] = 0;  // pairs this CTA merges at the end (at most its first and last): sflag[4..5]
+        for (int s = 0; s < NS; ++s) {
             mbar_init(smem_addr(&bars[s]), 1);
-            mbar_init(smem_addr(&bars[kStages + s]), C::NCW);
+            mbar_init(smem_addr(&bars[NS + s]), C::GW);
         }
         mbar_fence_init();
     }
     // rows past a short box are never written by TMA: keep them finite
     if (pa.deep_box < kTileRows || pa.ring_box < kTileRows) {
         uint4 *z = reinterpret_cast<uint4 *>(stages);
-        for (int i = tid; i < kStages * C::STAGE_BYTES / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid; i < NS * C::STAGE_BYTES / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
     }
+    // ---- per-sequence tile counts and their prefix sums (T is written by earlier kernels)
+    pdl_wait();
+    for (int n = tid; n < N; n += blockDim.x) {
+        const int T = a.T[n];
+        Ts[n] = T;
+        cum[n + 1] = seq_geom(T, pa).total * kvH;
+    }
+    if (tid == 0) cum[0] = 0;
     __syncthreads();
     if (warp == 0) {  // inclusive scan of cum[1..N] in chunks of 32
         int carry = 0;
@@ -145,39 +169,46 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     }
     __syncthreads();
 
+    pdl_trigger();  // the next kernel may be scheduled; it waits for this one to finish
     const int total = cum[N];
-    const int chunk = cdiv(total, static_cast<int>(gridDim.x));
+    int chunk = cdiv(total, static_cast<int>(gridDim.x));
+    if (chunk < a.min_chunk) chunk = a.min_chunk;
     const int g_begin = blockIdx.x * chunk;
     const int g_end = min(total, g_begin + chunk);
     if (g_begin >= g_end) return;
+    const int ntiles = g_end - g_begin;
 
     const uint32_t full0 = smem_addr(&bars[0]);
-    const uint32_t empty0 = smem_addr(&bars[kStages]);
+    const uint32_t empty0 = smem_addr(&bars[NS]);
     const uint32_t stage0 = smem_addr(stages);
 
     if (warp == C::NCW) {
         // ================================================================ producer
         if (lane == 0) {
-            tma_prefetch_desc(&tmKd); tma_prefetch_desc(&tmVd);
-            tma_prefetch_desc(&tmKw); tma_prefetch_desc(&tmVw);
-            TileIter it;
-            it.cum = cum; it.Ts = Ts;
-            it.start(g_begin, N, kvH, pa);
+            int n = seq_of(cum, N, g_begin);
+            SeqGeom sg = seq_geom(Ts[n], pa);
+            int rel = g_begin - cum[n];
+            int kh = rel / sg.total;
+            int lt = rel - kh * sg.total;
+            const int P0 = n * kvH + kh;
             int i = 0;
             bool ok = true;
-            for (int gt = g_begin; gt < g_end; ++gt, ++i) {
-                const int s = i % kStages;
-                if (i >= kStages && !mbar_wait_bounded(empty0 + 8 * s, ((i / kStages) - 1) & 1)) {
+            for (; i < ntiles; ++i) {
+                const int s = i % NS;
+                if (i >= NS && !mbar_wait_bounded(empty0 + 8 * s, ((i / NS) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                const Tile t = tile_at(it.s, it.lt, pa);
+                const Tile t = tile_at(sg, lt, pa);
                 const bool deep = t.kind == kDeep;
                 const int rows = deep ? pa.deep_box : pa.ring_box;
                 const CUtensorMap *mk = deep ? &tmKd : &tmKw;
                 const CUtensorMap *mv = deep ? &tmVd : &tmVw;
-                const int z = deep ? ((a.layer * N + it.n) * kvH + it.kh)
-                                   : (((a.layer * N + it.n) * a.R + t.plane) * kvH + it.kh);
+                const int z = deep ? ((a.layer * N + n) * kvH + kh)
+                                   : (((a.layer * N + n) * a.R + t.plane) * kvH + kh);
+                TileDesc &dsc = sdesc[s];
+                dsc.pair = n * kvH + kh; dsc.n = n; dsc.kh = kh; dsc.T = sg.T;
+                dsc.kind = t.kind; dsc.t0 = t.t0; dsc.cnt = t.cnt;
                 const uint32_t fb = full0 + 8 * s;
                 mbar_expect_tx(fb, 2 * C::NBOX * rows * 64);
                 const uint32_t kdst = stage0 + s * C::STAGE_BYTES;
@@ -187,94 +218,142 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     tma_load_3d(kdst + b * kBoxBytes, mk, fb, b * kBoxCols, t.y, z);
                     tma_load_3d(vdst + b * kBoxBytes, mv, fb, b * kBoxCols, t.y, z);
                 }
-                it.next(N, kvH, pa);
+                if (++lt == sg.total) {
+                    lt = 0;
+                    if (++kh == kvH) {
+                        kh = 0;
+                        if (++n < N) sg = seq_geom(Ts[n], pa);
+                    }
+                }
+                if (i == NS - 1) {  // pipeline full: warm L2 with the query rows of the later pairs
+                    const int p_last = pair_of(cum, N, kvH, g_end - 1);
+                    for (int p = P0 + 1; p <= p_last; ++p) {
+                        const int pn = p / kvH, pk = p - pn * kvH;
+                        for (int j = 0; j < a.B; ++j) {
+                            const char *row = reinterpret_cast<const char *>(
+                                a.q + ((static_cast<size_t>(pn) * a.B + j) * a.Hq + pk * a.g) * D);
+                            for (int off = 0; off < a.g * D * 2; off += 128)
+                                asm volatile("prefetch.global.L2 [%0];" ::"l"(row + off));
+                        }
+                    }
+                }
             }
             if (!ok) {
                 atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
                 // drain: the last issue of every stage must land before the CTA exits
-                for (int k = (i > kStages ? i - kStages : 0); k < i; ++k)
-                    mbar_wait_bounded(full0 + 8 * (k % kStages), (k / kStages) & 1);
+                for (int k = (i > NS ? i - NS : 0); k < i; ++k)
+                    mbar_wait_bounded(full0 + 8 * (k % NS), (k / NS) & 1);
             }
         }
-        // the producer warp takes part in no consumer barrier (id 1)
-        return;
+        return;  // the producer warp takes part in no consumer barrier (id 1)
     }
 
     // ==================================================================== consumers
-    const int rg = warp / C::WK;   // row group: query rows 16*rg .. 16*rg + 15
-    const int kg = warp % C::WK;   // key group: 16-key sub-blocks kg, kg + WK, ...
+    const int tg = warp / C::GW;             // tile group: tiles i with i % TG == tg
+    const int rg = (warp % C::GW) / WK;      // row group: queries NQ*rg .. NQ*rg + NQ-1
+    const int kg = warp % WK;                // key group: sub-blocks kg*SB .. kg*SB + SB-1
     const int g4 = lane >> 2, c4 = lane & 3;
-    const int ctid = tid;          // consumers are threads 0 .. NCW*32 - 1
     const int nct = C::NCW * 32;
 
-    // query rows held by this thread: i = 16*rg + g4 (+8); row i is block position i / g
-    int jrow[2];
-    bool rvalid[2];
+    // query columns held by this thread: q = NQ*rg + 8*nq + 2*c4 + e  (e = 0, 1)
+    int jq[NQT][2];
+    bool qvalid[NQT][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int i = 16 * rg + g4 + 8 * h;
-        rvalid[h] = i < a.Mq;
-        jrow[h] = rvalid[h] ? i / a.g : a.B - 1;
-    }
+    for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int i = C::NQ * rg + 8 * nq + 2 * c4 + e;
+            qvalid[nq][e] = i < a.Mq;
+            jq[nq][e] = qvalid[nq][e] ? i / a.g : a.B - 1;
+        }
     // ldmatrix lane geometry (64-byte swizzle: 16-byte chunk ^= (row >> 1) & 3)
     const int mi = lane >> 3, r8 = lane & 7;
     const uint32_t swz = static_cast<uint32_t>(r8 >> 1);
-    const int krow_off = (mi >> 1) * 8 + r8;  // K: matrices (keys 0-7 | 8-15) x (d lo | hi)
-    const uint32_t kcol_sel = mi & 1;
-    const int vrow_off = (mi & 1) * 8 + r8;   // V (trans): (keys 0-7 | 8-15) x (dv lo | hi)
-    const uint32_t vcol_sel = mi >> 1;
+    const uint32_t krow_off = static_cast<uint32_t>((mi & 1) * 8 + r8);  // K as A: (keys lo|hi) x (d lo|hi)
+    const uint32_t kcol_sel = static_cast<uint32_t>(mi >> 1);
+    const uint32_t vrow_off = static_cast<uint32_t>((mi >> 1) * 8 + r8); // V^T as A: (dv lo|hi) x (keys lo|hi)
+    const uint32_t vcol_sel = static_cast<uint32_t>(mi & 1);
 
-    float o[D / 8][4];
-    float m_run[2], l_run[2];
-    uint32_t qa[D / 16][4];
+    float o[D / 16][NQT][4];
+    float m_ref[NQT][2], l_run[NQT][2];
+    uint32_t qb[D / 16][NQT][2];
 
-    TileIter it;
-    it.cum = cum; it.Ts = Ts;
-    it.start(g_begin, N, kvH, pa);
-    int cur_pair = -1, cur_n = 0, cur_kh = 0;
+    const int P_first = pair_of(cum, N, kvH, g_begin);
+    const int P_last = pair_of(cum, N, kvH, g_end - 1);
+    int fin_next = P_first;  // next pair to finalize (every consumer warp finalizes each pair once)
+    int st_pair = -1;        // pair whose partial state this warp holds
     bool aborted = false;
+
+    auto reset_state = [&]() {
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+            for (int nq = 0; nq < NQT; ++nq) o[mt][nq][0] = o[mt][nq][1] = o[mt][nq][2] = o[mt][nq][3] = 0.f;
+#pragma unroll
+        for (int nq = 0; nq < NQT; ++nq) {
+            m_ref[nq][0] = m_ref[nq][1] = -INFINITY;
+            l_run[nq][0] = l_run[nq][1] = 0.f;
+        }
+    };
 
     auto load_q = [&](int n, int kh) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int i = 16 * rg + g4 + 8 * h;
+        for (int nq = 0; nq < NQT; ++nq) {
+            const int i = C::NQ * rg + 8 * nq + g4;  // B-operand column = query g4 of the tile
             const uint32_t *qp = nullptr;
-            if (rvalid[h]) {
-                const int j = i / a.g, hg = i - (i / a.g) * a.g;
+            if (i < a.Mq) {
+                const int j = i / a.g, hg = i - j * a.g;
                 qp = reinterpret_cast<const uint32_t *>(
                     a.q + ((static_cast<size_t>(n) * a.B + j) * a.Hq + kh * a.g + hg) * D);
             }
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
-                qa[ks][h] = qp ? __ldg(qp + (16 * ks + 2 * c4) / 2) : 0u;
-                qa[ks][2 + h] = qp ? __ldg(qp + (16 * ks + 8 + 2 * c4) / 2) : 0u;
+                qb[ks][nq][0] = qp ? __ldg(qp + 8 * ks + c4) : 0u;
+                qb[ks][nq][1] = qp ? __ldg(qp + 8 * ks + 4 + c4) : 0u;
             }
         }
-#pragma unroll
-        for (int nt = 0; nt < D / 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-        m_run[0] = m_run[1] = -INFINITY;
-        l_run[0] = l_run[1] = 0.f;
     };
 
-    auto finalize = [&](int n, int kh) {
-        const int P = n * kvH + kh;
-        // complete the row sums over the quad
+    // ---------------------------------------------------------------- finalize one pair
+    auto finalize = [&](int p, bool have) {
+        const int n = p / kvH, kh = p - (p / kvH) * kvH;
+        float *mw = mo + warp * C::NQ * C::DP;
+        if (have) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
-            l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
-        }
-        float *mw = mo + warp * 16 * D;
+            for (int nq = 0; nq < NQT; ++nq)
 #pragma unroll
-        for (int nt = 0; nt < D / 8; ++nt) {
-            *reinterpret_cast<float2 *>(&mw[g4 * D + 8 * nt + 2 * c4]) = make_float2(o[nt][0], o[nt][1]);
-            *reinterpret_cast<float2 *>(&mw[(g4 + 8) * D + 8 * nt + 2 * c4]) = make_float2(o[nt][2], o[nt][3]);
-        }
-        if (c4 == 0) {
-            mml[(warp * 16 + g4) * 2] = m_run[0];
-            mml[(warp * 16 + g4) * 2 + 1] = l_run[0];
-            mml[(warp * 16 + g4 + 8) * 2] = m_run[1];
-            mml[(warp * 16 + g4 + 8) * 2 + 1] = l_run[1];
+                for (int e = 0; e < 2; ++e) {
+                    float l = l_run[nq][e];
+                    l += __shfl_xor_sync(0xffffffffu, l, 4);
+                    l += __shfl_xor_sync(0xffffffffu, l, 8);
+                    l += __shfl_xor_sync(0xffffffffu, l, 16);
+                    l_run[nq][e] = l;
+                }
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                for (int nq = 0; nq < NQT; ++nq) {
+                    const int q0 = 8 * nq + 2 * c4;
+                    mw[q0 * C::DP + 16 * mt + g4] = o[mt][nq][0];
+                    mw[(q0 + 1) * C::DP + 16 * mt + g4] = o[mt][nq][1];
+                    mw[q0 * C::DP + 16 * mt + 8 + g4] = o[mt][nq][2];
+                    mw[(q0 + 1) * C::DP + 16 * mt + 8 + g4] = o[mt][nq][3];
+                }
+            if (g4 == 0) {
+#pragma unroll
+                for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int q = 8 * nq + 2 * c4 + e;
+                        mml[(warp * C::NQ + q) * 2] = m_ref[nq][e];
+                        mml[(warp * C::NQ + q) * 2 + 1] = l_run[nq][e];
+                    }
+            }
+        } else {
+            for (int q = lane; q < C::NQ; q += 32) {
+                mml[(warp * C::NQ + q) * 2] = -INFINITY;
+                mml[(warp * C::NQ + q) * 2 + 1] = 0.f;
+            }
         }
         named_bar_sync(1, nct);
         const bool abort_now = *reinterpret_cast<volatile int *>(&sflag[1]) != 0;
@@ -283,207 +362,329 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         const int c_first = start / chunk, c_last = (start + tot_n - 1) / chunk;
         const int nparts = c_last - c_first + 1;
         const bool sole = nparts == 1;
-        const int rows = WR * 16;
-        for (int e = ctid; e < rows * D; e += nct) {
-            const int i = e / D, col = e - (e / D) * D;
-            const int rgi = i >> 4, row = i & 15;
+        // per query row: the maximum over the warps that saw it, their weights and the sum
+        for (int i = tid; i < C::ROWS; i += nct) {
+            const int rgi = i / C::NQ, q = i - rgi * C::NQ;
             float M = -INFINITY;
 #pragma unroll
-            for (int k = 0; k < C::WK; ++k) M = fmaxf(M, mml[((rgi * C::WK + k) * 16 + row) * 2]);
-            float acc = 0.f, L = 0.f;
-            if (M != -INFINITY) {
+            for (int t2 = 0; t2 < TG; ++t2)
 #pragma unroll
-                for (int k = 0; k < C::WK; ++k) {
-                    const int w = rgi * C::WK + k;
-                    const float mk = mml[(w * 16 + row) * 2];
-                    if (mk != -INFINITY) {
-                        const float f = exp2f(mk - M);
-                        acc += mo[(w * 16 + row) * D + col] * f;
-                        L += mml[(w * 16 + row) * 2 + 1] * f;
-                    }
+                for (int k = 0; k < WK; ++k) M = fmaxf(M, mml[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * 2]);
+            float L = 0.f;
+#pragma unroll
+            for (int t2 = 0; t2 < TG; ++t2)
+#pragma unroll
+                for (int k = 0; k < WK; ++k) {
+                    const int w = t2 * C::GW + rgi * WK + k;
+                    const float mk = mml[(w * C::NQ + q) * 2];
+                    const float f = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                    wq[i * (TG * WK) + t2 * WK + k] = f;
+                    L += f * mml[(w * C::NQ + q) * 2 + 1];
                 }
-            }
-            if (abort_now) continue;
+            fin[i * 2] = M;
+            fin[i * 2 + 1] = L;
+        }
+        named_bar_sync(1, nct);
+        const int rows = sole ? a.Mq : C::ROWS;
+        for (int e = tid; e < rows * D && !abort_now; e += nct) {
+            const int i = e / D, col = e - i * D;
+            const int rgi = i / C::NQ, q = i - rgi * C::NQ;
+            float acc = 0.f;
+#pragma unroll
+            for (int t2 = 0; t2 < TG; ++t2)
+#pragma unroll
+                for (int k = 0; k < WK; ++k) {
+                    // a warp that saw no key of this row left its slice of the buffer stale
+                    const float w = wq[i * (TG * WK) + t2 * WK + k];
+                    if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
+                }
             if (sole) {
-                if (i < a.Mq) {
-                    const int j = i / a.g, h = kh * a.g + (i - j * a.g);
-                    const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
-                    a.out[orow * D + col] = __float2bfloat16_rn(acc / L);
-                    if (col == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
-                }
+                const int j = i / a.g, h = kh * a.g + (i - j * a.g);
+                const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
+                a.out[orow * D + col] = __float2bfloat16_rn(acc / fin[i * 2 + 1]);
+                if (col == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
             } else {
-                const size_t prow = (static_cast<size_t>(blockIdx.x) + P) * a.part_rows + i;
+                const size_t prow = (static_cast<size_t>(blockIdx.x) + p) * C::ROWS + i;
                 a.part_o[prow * D + col] = acc;
                 if (col == 0) {
-                    a.part_ml[prow * 2] = M;
-                    a.part_ml[prow * 2 + 1] = L;
+                    a.part_ml[prow * 2] = fin[i * 2];
+                    a.part_ml[prow * 2 + 1] = fin[i * 2 + 1];
                 }
             }
         }
-        if (!sole && !abort_now) {
+        named_bar_sync(1, nct);  // partials written; the merge buffer is free again
+        if (!sole && !abort_now && tid == 0) {
+            // publish this CTA's partial (bar.sync + one fence covers every thread's writes)
             __threadfence();
-            named_bar_sync(1, nct);
-            if (ctid == 0) {
-                const int old = atomicAdd(&a.counters[P], 1);
-                sflag[0] = (old == nparts - 1) ? 1 : 0;
-            }
-            named_bar_sync(1, nct);
-            if (sflag[0]) {
+            const int old = atomicAdd(&a.counters[p], 1);
+            if (old == nparts - 1) {
                 __threadfence();
-                for (int e = ctid; e < a.Mq * D; e += nct) {
-                    const int i = e / D, col = e - (e / D) * D;
-                    float M = -INFINITY;
-                    for (int c = c_first; c <= c_last; ++c)
-                        M = fmaxf(M, __ldcg(&a.part_ml[((static_cast<size_t>(c) + P) * a.part_rows + i) * 2]));
-                    float acc = 0.f, L = 0.f;
-                    for (int c = c_first; c <= c_last; ++c) {
-                        const size_t prow = (static_cast<size_t>(c) + P) * a.part_rows + i;
-                        const float mk = __ldcg(&a.part_ml[prow * 2]);
-                        if (mk != -INFINITY) {
-                            const float f = exp2f(mk - M);
-                            acc += __ldcg(&a.part_o[prow * D + col]) * f;
-                            L += __ldcg(&a.part_ml[prow * 2 + 1]) * f;
-                        }
-                    }
-                    const int j = i / a.g, h = kh * a.g + (i - j * a.g);
-                    const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
-                    a.out[orow * D + col] = __float2bfloat16_rn(acc / L);
-                    if (col == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
-                }
-                if (ctid == 0) a.counters[P] = 0;
+                sflag[4 + sflag[3]] = p;  // merged at the end of this CTA's tiles
+                sflag[3] += 1;
             }
         }
-        named_bar_sync(1, nct);  // the merge buffer is rewritten by the next pair
     };
 
-    int i = 0;
-    for (int gt = g_begin; gt < g_end; ++gt, ++i) {
-        const int P = it.n * kvH + it.kh;
-        if (P != cur_pair) {
-            if (cur_pair >= 0) finalize(cur_n, cur_kh);
-            cur_pair = P; cur_n = it.n; cur_kh = it.kh;
-            load_q(cur_n, cur_kh);
+    // ---------------------------------------------------------------- merge the partials of one pair
+    // Runs in the CTA that arrived last, after all of its own tiles (the stage buffers are free).
+    auto merge_pair = [&](int p) {
+        const int n = p / kvH, kh = p - (p / kvH) * kvH;
+        const int tot_n = (cum[n + 1] - cum[n]) / kvH;
+        const int start = cum[n] + kh * tot_n;
+        const int c_first = start / chunk, c_last = (start + tot_n - 1) / chunk;
+        const int nparts = c_last - c_first + 1;
+        float *pw = reinterpret_cast<float *>(stages);  // [nparts][ROWS] m, then weights
+        float *pl = pw + nparts * C::ROWS;              // [nparts][ROWS] l
+        float *rowML = fin;                             // [ROWS][2] final M, L
+        for (int e = tid; e < nparts * a.Mq; e += nct) {
+            const int c = e / a.Mq, i = e - (e / a.Mq) * a.Mq;
+            const size_t prow = (static_cast<size_t>(c_first + c) + p) * C::ROWS + i;
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(&a.part_ml[prow * 2]));
+            pw[c * C::ROWS + i] = ml.x;
+            pl[c * C::ROWS + i] = ml.y;
         }
-        const int s = i % kStages;
-        if (!aborted && !mbar_wait_bounded(full0 + 8 * s, (i / kStages) & 1)) {
-            aborted = true;
-            atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
-            *reinterpret_cast<volatile int *>(&sflag[1]) = 1;
+        named_bar_sync(1, nct);
+        for (int i = tid; i < a.Mq; i += nct) {
+            float M = -INFINITY;
+            for (int c = 0; c < nparts; ++c) M = fmaxf(M, pw[c * C::ROWS + i]);
+            float L = 0.f;
+            for (int c = 0; c < nparts; ++c) {
+                const float mk = pw[c * C::ROWS + i];
+                const float w = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                pw[c * C::ROWS + i] = w;
+                L += w * pl[c * C::ROWS + i];
+            }
+            rowML[i * 2] = M;
+            rowML[i * 2 + 1] = L;
         }
-        if (!aborted) {
-            const Tile t = tile_at(it.s, it.lt, pa);
-            const int T = it.s.T;
-            const uint32_t kbase = stage0 + s * C::STAGE_BYTES;
-            const uint32_t vbase = kbase + C::NBOX * kBoxBytes;
+        named_bar_sync(1, nct);
+        for (int e = tid; e < a.Mq * (D / 4); e += nct) {
+            const int i = e / (D / 4), c4x = e - (e / (D / 4)) * (D / 4);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+            for (int c = 0; c < nparts; ++c) {
+                const float w = pw[c * C::ROWS + i];
+                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                    &a.part_o[((static_cast<size_t>(c_first + c) + p) * C::ROWS + i) * D + 4 * c4x]));
+                acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+            }
+            const float invL = 1.f / rowML[i * 2 + 1];
+            const int j = i / a.g, h = kh * a.g + (i - j * a.g);
+            const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
+            __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + 4 * c4x]);
+            op[0] = __floats2bfloat162_rn(acc.x * invL, acc.y * invL);
+            op[1] = __floats2bfloat162_rn(acc.z * invL, acc.w * invL);
+            if (c4x == 0 && a.lse)
+                a.lse[orow] = (rowML[i * 2] + __log2f(rowML[i * 2 + 1])) * 0.69314718055994531f;
+        }
+        if (tid == 0) a.counters[p] = 0;
+        named_bar_sync(1, nct);
+    };
+
+    // ---------------------------------------------------------------- one tile
+    auto compute = [&](const TileDesc &dsc, int s, auto fast_tag) {
+        constexpr bool FAST = decltype(fast_tag)::value;
+        const uint32_t kbase = stage0 + s * C::STAGE_BYTES;
+        const uint32_t vbase = kbase + C::NBOX * kBoxBytes;
+        float x[C::SB][NQT][4];
+        bool act[C::SB];
 #pragma unroll
-            for (int kb0 = 0; kb0 < 4 / C::WK; ++kb0) {
-                const int kb = kg + kb0 * C::WK;
-                if (16 * kb >= t.cnt) break;
-                // ---- S = Q K^T for 16 keys
-                float S[2][4];
+        for (int sb = 0; sb < C::SB; ++sb) {
+            const int kb = kg * C::SB + sb;
+            act[sb] = FAST || 16 * kb < dsc.cnt;
+            float se[NQT][4], so[NQT][4];
 #pragma unroll
-                for (int x = 0; x < 2; ++x) S[x][0] = S[x][1] = S[x][2] = S[x][3] = 0.f;
-                const uint32_t krow = static_cast<uint32_t>(16 * kb + krow_off);
+            for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) se[nq][e] = so[nq][e] = 0.f;
+            if (act[sb]) {
+                const uint32_t krow = static_cast<uint32_t>(16 * kb) + krow_off;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks) {
                     const uint32_t col16 = static_cast<uint32_t>(2 * (ks & 1)) + kcol_sel;
                     const uint32_t addr = kbase + (ks >> 1) * kBoxBytes + krow * 64 + ((col16 ^ swz) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4(addr, b0, b1, b2, b3);
-                    mma_16816(S[0], qa[ks], b0, b1);
-                    mma_16816(S[1], qa[ks], b2, b3);
-                }
-                // ---- mask, scale, online softmax (base 2)
-                float pr[2][4];
-                float mt[2] = {-INFINITY, -INFINITY};
+                    uint32_t af[4];
+                    ldsm_x4(addr, af[0], af[1], af[2], af[3]);
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int h = e >> 1;
-                        const int kk = 16 * kb + 8 * nt + 2 * c4 + (e & 1);
-                        const int tpos = t.t0 + kk;
-                        const int p = T + jrow[h];
-                        bool vis = kk < t.cnt;
-                        if (t.kind == kRing)
-                            vis = vis && tpos <= p && (pa.mode_eff != 0 || tpos >= T || tpos >= p - pa.W);
-                        else if (t.kind == kDual)
-                            vis = vis && tpos < p - pa.W;
-                        const float x = vis ? S[nt][e] * a.scale_log2 : -INFINITY;
-                        pr[nt][e] = x;
-                        mt[h] = fmaxf(mt[h], x);
+                    for (int nq = 0; nq < NQT; ++nq) {
+                        if (ks & 1) mma_16816(so[nq], af, qb[ks][nq][0], qb[ks][nq][1]);
+                        else mma_16816(se[nq], af, qb[ks][nq][0], qb[ks][nq][1]);
                     }
-                float alpha[2];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 1));
-                    mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], 2));
-                    const float mn = fmaxf(m_run[h], mt[h]);
-                    alpha[h] = (mn == -INFINITY) ? 1.f : exp2f(m_run[h] - mn);
-                    m_run[h] = mn;
-                }
-                uint32_t pa_frag[4];
-                float lsum[2] = {0.f, 0.f};
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const float mn = m_run[hh];
-                        const float p0 = (mn == -INFINITY) ? 0.f : exp2f(pr[nt][2 * hh] - mn);
-                        const float p1 = (mn == -INFINITY) ? 0.f : exp2f(pr[nt][2 * hh + 1] - mn);
-                        const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                        const float2 pf = __bfloat1622float2(pb);
-                        lsum[hh] += pf.x + pf.y;
-                        pa_frag[2 * nt + hh] = *reinterpret_cast<const uint32_t *>(&pb);
-                    }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) l_run[h] = l_run[h] * alpha[h] + lsum[h];
-#pragma unroll
-                for (int nt = 0; nt < D / 8; ++nt) {
-                    o[nt][0] *= alpha[0]; o[nt][1] *= alpha[0];
-                    o[nt][2] *= alpha[1]; o[nt][3] *= alpha[1];
-                }
-                // ---- O += P V for 16 keys
-                const uint32_t vrow = static_cast<uint32_t>(16 * kb + vrow_off);
-#pragma unroll
-                for (int dv = 0; dv < D / 16; ++dv) {
-                    const uint32_t col16 = static_cast<uint32_t>(2 * (dv & 1)) + vcol_sel;
-                    const uint32_t addr = vbase + (dv >> 1) * kBoxBytes + vrow * 64 + ((col16 ^ swz) << 4);
-                    uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(addr, b0, b1, b2, b3);
-                    mma_16816(o[2 * dv], pa_frag, b0, b1);
-                    mma_16816(o[2 * dv + 1], pa_frag, b2, b3);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty0 + 8 * s);
+#pragma unroll
+            for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v = (se[nq][e] + so[nq][e]) * a.scale_log2;
+                    if (!FAST) {
+                        const int kk = 16 * kb + g4 + 8 * (e >> 1);
+                        const int tpos = dsc.t0 + kk;
+                        const int pq = dsc.T + jq[nq][e & 1];
+                        bool vis = act[sb] && kk < dsc.cnt;
+                        if (dsc.kind == kRing)
+                            vis = vis && tpos <= pq && (pa.mode_eff != 0 || tpos >= dsc.T || tpos >= pq - pa.W);
+                        else if (dsc.kind == kDual)
+                            vis = vis && tpos < pq - pa.W;
+                        v = vis ? v : -INFINITY;
+                    }
+                    x[sb][nq][e] = v;
+                }
         }
-        it.next(N, kvH, pa);
+        // column maxima over this warp's keys, then over the 8 lanes sharing a column
+        float alpha[NQT][2];
+        bool need = false;
+#pragma unroll
+        for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float mt = -INFINITY;
+#pragma unroll
+                for (int sb = 0; sb < C::SB; ++sb) mt = fmaxf(mt, fmaxf(x[sb][nq][e], x[sb][nq][e + 2]));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                alpha[nq][e] = 1.f;
+                if (mt > m_ref[nq][e] + kLazyMax) {  // also true when m_ref is -inf and mt is finite
+                    alpha[nq][e] = exp2f(m_ref[nq][e] - mt);
+                    m_ref[nq][e] = mt;
+                    need = true;
+                }
+            }
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int nq = 0; nq < NQT; ++nq) {
+                l_run[nq][0] *= alpha[nq][0];
+                l_run[nq][1] *= alpha[nq][1];
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    o[mt][nq][0] *= alpha[nq][0]; o[mt][nq][1] *= alpha[nq][1];
+                    o[mt][nq][2] *= alpha[nq][0]; o[mt][nq][3] *= alpha[nq][1];
+                }
+            }
+        }
+        // P^T fragments: rows (keys) g4 / g4+8, columns (queries) 2c4, 2c4+1 -> movmatrix
+#pragma unroll
+        for (int sb = 0; sb < C::SB; ++sb) {
+            if (!act[sb]) continue;
+            const int kb = kg * C::SB + sb;
+            uint32_t pb[NQT][2];
+#pragma unroll
+            for (int nq = 0; nq < NQT; ++nq) {
+                const float r0 = m_ref[nq][0], r1 = m_ref[nq][1];
+                const float p0 = (r0 == -INFINITY) ? 0.f : exp2f(x[sb][nq][0] - r0);
+                const float p1 = (r1 == -INFINITY) ? 0.f : exp2f(x[sb][nq][1] - r1);
+                const float p2 = (r0 == -INFINITY) ? 0.f : exp2f(x[sb][nq][2] - r0);
+                const float p3 = (r1 == -INFINITY) ? 0.f : exp2f(x[sb][nq][3] - r1);
+                const __nv_bfloat162 lo = __floats2bfloat162_rn(p0, p1);
+                const __nv_bfloat162 hi = __floats2bfloat162_rn(p2, p3);
+                const float2 flo = __bfloat1622float2(lo), fhi = __bfloat1622float2(hi);
+                l_run[nq][0] += flo.x + fhi.x;
+                l_run[nq][1] += flo.y + fhi.y;
+                pb[nq][0] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&lo));
+                pb[nq][1] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&hi));
+            }
+            // O^T += V^T P^T
+            const uint32_t vrow = static_cast<uint32_t>(16 * kb) + vrow_off;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                const uint32_t col16 = static_cast<uint32_t>(2 * (mt & 1)) + vcol_sel;
+                const uint32_t addr = vbase + (mt >> 1) * kBoxBytes + vrow * 64 + ((col16 ^ swz) << 4);
+                uint32_t af[4];
+                ldsm_x4_t(addr, af[0], af[1], af[2], af[3]);
+#pragma unroll
+                for (int nq = 0; nq < NQT; ++nq) mma_16816(o[mt][nq], af, pb[nq][0], pb[nq][1]);
+            }
+        }
+    };
+
+    reset_state();
+    for (int i = tg; i < ntiles; i += TG) {
+        const int s = i % NS;
+        if (!mbar_wait_bounded(full0 + 8 * s, (i / NS) & 1)) {
+            aborted = true;
+            atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
+            *reinterpret_cast<volatile int *>(&sflag[1]) = 1;
+            break;
+        }
+        const TileDesc dsc = sdesc[s];
+        if (dsc.pair != st_pair) {
+            while (fin_next < dsc.pair) {
+                finalize(fin_next, st_pair == fin_next);
+                ++fin_next;
+            }
+            st_pair = dsc.pair;
+            reset_state();
+            load_q(dsc.n, dsc.kh);
+        }
+        if (dsc.kind == kDeep && dsc.cnt == kTileRows)
+            compute(dsc, s, std::integral_constant<bool, true>());
+        else
+            compute(dsc, s, std::integral_constant<bool, false>());
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * s);
     }
-    if (cur_pair >= 0) finalize(cur_n, cur_kh);
+    while (fin_next <= P_last) {
+        finalize(fin_next, !aborted && st_pair == fin_next);
+        ++fin_next;
+    }
+    named_bar_sync(1, nct);
+    if (*reinterpret_cast<volatile int *>(&sflag[1]) == 0) {
+        const int nm = sflag[3];
+        for (int k = 0; k < nm; ++k) merge_pair(sflag[4 + k]);
+    }
 }
 
-template <int D, int WR>
-static cudaError_t set_attr_one(int N) {
-    return cudaFuncSetAttribute(ripe_verify_kernel<D, WR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                verify_smem_bytes(D, WR, N));
+// ---------------------------------------------------------------- host side
+template <int D, int NQT, int WR, int WK, int TG>
+struct Inst {
+    using C = VCfg<D, NQT, WR, WK, TG>;
+    static cudaError_t set_attr(int N) {
+        return cudaFuncSetAttribute(ripe_verify_kernel<D, NQT, WR, WK, TG>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for<C>(N));
+    }
+    static void launch(const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
+        launch_pdl(ripe_verify_kernel<D, NQT, WR, WK, TG>, dim3(grid), dim3(C::THREADS),
+                   smem_bytes_for<C>(c->N), s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
+    }
+};
+
+// query-side configuration by the number of query rows per kv head (B * group)
+//   <= 8  : one 8-query tile per warp, 2 tile groups of 4 warps
+//   <= 16 : two 8-query tiles per warp, 2 tile groups of 4 warps
+//   <= 32 : two row groups x 4 key groups
+//   <= 64 : four row groups x 2 key groups (32 keys per warp per tile)
+#define RIPE_QCFG_LIST(D)                                                          \
+    Inst<D, 1, 1, 4, 2>, Inst<D, 2, 1, 4, 2>, Inst<D, 2, 2, 4, 1>, Inst<D, 2, 4, 2, 1>
+
+static int qcfg_of(int Mq) { return Mq <= 8 ? 0 : Mq <= 16 ? 1 : Mq <= 32 ? 2 : 3; }
+
+template <class... I>
+static cudaError_t set_all(int N) {
+    cudaError_t e = cudaSuccess;
+    ((e = (e == cudaSuccess ? I::set_attr(N) : e)), ...);
+    return e;
 }
 
 int set_verify_attributes(int d, int N) {
-    cudaError_t e = cudaSuccess;
+    cudaError_t e;
     switch (d) {
-        case 64: e = set_attr_one<64, 1>(N); if (!e) e = set_attr_one<64, 2>(N); if (!e) e = set_attr_one<64, 4>(N); break;
-        case 96: e = set_attr_one<96, 1>(N); if (!e) e = set_attr_one<96, 2>(N); if (!e) e = set_attr_one<96, 4>(N); break;
-        case 128: e = set_attr_one<128, 1>(N); if (!e) e = set_attr_one<128, 2>(N); if (!e) e = set_attr_one<128, 4>(N); break;
+        case 64: e = set_all<RIPE_QCFG_LIST(64)>(N); break;
+        case 96: e = set_all<RIPE_QCFG_LIST(96)>(N); break;
+        case 128: e = set_all<RIPE_QCFG_LIST(128)>(N); break;
         default: return RIPE_EINVAL;
     }
     return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 
-template <int D, int WR>
-static void launch_one(const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
-    ripe_verify_kernel<D, WR><<<grid, VCfg<D, WR>::THREADS, verify_smem_bytes(D, WR, c->N), s>>>(
-        c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
+template <class I0, class I1, class I2, class I3>
+static void launch_d(int qc, const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
+    switch (qc) {
+        case 0: I0::launch(c, grid, a, s); break;
+        case 1: I1::launch(c, grid, a, s); break;
+        case 2: I2::launch(c, grid, a, s); break;
+        default: I3::launch(c, grid, a, s); break;
+    }
 }
 
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,
@@ -514,28 +715,23 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
     a.R = c->R;
     a.layer = layer;
     a.Mq = c->B_cur * c->g;
-    const int wr = a.Mq <= 16 ? 1 : (a.Mq <= 32 ? 2 : 4);
-    a.part_rows = 16 * wr;
+    a.min_chunk = RIPE_MIN_CHUNK;  // bounds the number of partials of one (sequence, kv head)
     a.scale_log2 = scale * 1.4426950408889634f;
+    const int qc = qcfg_of(a.Mq);
 
     // grid: one CTA per SM, fewer when the host copy of T says there is less work
-    int grid = c->num_sms;
+    int grid = c->num_sms < 256 ? c->num_sms : 256;  // the last-CTA merge keeps <= 256 partial weights per row
     if (c->synced) {
         long total = 0;
         for (int n = 0; n < c->N; ++n) total += static_cast<long>(seq_geom(c->T[n], a.plan).total) * c->kvH;
-        if (total < grid) grid = static_cast<int>(total);
+        const long need = (total + a.min_chunk - 1) / a.min_chunk;
+        if (need < grid) grid = static_cast<int>(need);
     }
     if (grid < 1) grid = 1;
-    switch (c->d * 8 + wr) {
-        case 64 * 8 + 1: launch_one<64, 1>(c, grid, a, s); break;
-        case 64 * 8 + 2: launch_one<64, 2>(c, grid, a, s); break;
-        case 64 * 8 + 4: launch_one<64, 4>(c, grid, a, s); break;
-        case 96 * 8 + 1: launch_one<96, 1>(c, grid, a, s); break;
-        case 96 * 8 + 2: launch_one<96, 2>(c, grid, a, s); break;
-        case 96 * 8 + 4: launch_one<96, 4>(c, grid, a, s); break;
-        case 128 * 8 + 1: launch_one<128, 1>(c, grid, a, s); break;
-        case 128 * 8 + 2: launch_one<128, 2>(c, grid, a, s); break;
-        case 128 * 8 + 4: launch_one<128, 4>(c, grid, a, s); break;
+    switch (c->d) {
+        case 64: launch_d<RIPE_QCFG_LIST(64)>(qc, c, grid, a, s); break;
+        case 96: launch_d<RIPE_QCFG_LIST(96)>(qc, c, grid, a, s); break;
+        case 128: launch_d<RIPE_QCFG_LIST(128)>(qc, c, grid, a, s); break;
         default: return RIPE_EINVAL;
     }
     c->launches += 1;
