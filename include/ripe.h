@@ -49,7 +49,8 @@ enum ripe_status {
     RIPE_ENOMEM = -2,    /* device or host allocation failed */
     RIPE_ECAPACITY = -3, /* committed + block positions would exceed max_T */
     RIPE_ESTATE = -4,    /* call out of order (e.g. verify before the plane was appended) */
-    RIPE_ECUDA = -5      /* a CUDA runtime call or kernel launch failed */
+    RIPE_ECUDA = -5,     /* a CUDA runtime call or kernel launch failed */
+    RIPE_ESCRATCH = -6   /* the allocation-free entry point's static scratch is too small */
 };
 
 /* How the window of full-depth positions is measured for a query at position p = T + j.
@@ -185,6 +186,46 @@ int ripe_cache_export(ripe_cache_t *c, int n, int layer, void *k_out, void *v_ou
 
 /* Read and clear the device error word (synchronises `stream`); *err_out gets its bits. */
 int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream);
+
+/*
+ * Allocation-free verification attention.  The paper has no counterpart: this entry point
+ * exists for callers that cannot call cudaMalloc -- code whose device memory belongs to
+ * someone else (an inference engine's memory pool, a framework that preallocates all device
+ * memory) or code running while a stream capture is open, where allocation is not allowed.
+ * It computes exactly what ripe_verify_attn computes, over cache buffers that the caller
+ * owns and has filled in the documented layout, and allocates nothing.
+ *
+ * Its scratch (partial results of the split key ranges and their arrival counters) is one
+ * file-scope device array of RIPE_STATIC_SCRATCH_BYTES, which every GPU that loads the
+ * library holds until the process exits.  A problem whose scratch would exceed it is rejected
+ * with RIPE_ESCRATCH: it needs (S + batch * kv_heads) * rows * (head_dim + 2) * 4 bytes plus
+ * batch * kv_heads * 4, where S is the number of SMs and rows is 8, 16, 32 or 64 (the block
+ * length times q_heads / kv_heads, rounded up to one of those).
+ *
+ * The first call on a device sets up that device (looks up the array's device address and
+ * the SM count) with the device current; make that first call before any stream capture.
+ * Every call shares the array and it keeps the last call's contents; the counters are
+ * cleared on `stream` at each call.  Calls that overlap on the GPU (other streams, or other
+ * host threads) race on the array and must be serialised by the caller.
+ * The view's buffers must stay valid until the work enqueued on `stream` has finished.
+ * `device_error` (device uint32, optional) receives RIPE_DEVERR_* bits; the caller clears it.
+ */
+#define RIPE_STATIC_SCRATCH_BYTES (4u << 20)
+
+typedef struct ripe_cache_view {
+    int32_t batch, layers, q_heads, kv_heads, head_dim, loops; /* as for ripe_cache_alloc */
+    int32_t window, max_T, max_B, window_mode;                  /* as for ripe_cache_alloc */
+    int32_t block_len;       /* B of the block being verified (1 .. max_B) */
+    const void *k_deep;      /* bf16 [layers][batch][kv_heads][max_T - W][head_dim], NULL when W >= max_T */
+    const void *v_deep;
+    const void *k_ring;      /* bf16 [layers][batch][loops][kv_heads][S][head_dim], S = min(W + max_B, max_T),
+                                position t at slot t mod S */
+    const void *v_ring;
+    const int32_t *lengths;  /* device int32 [batch]: committed positions T_n */
+} ripe_cache_view;
+
+int ripe_verify_attn_static(const ripe_cache_view *view, int layer, int r, const void *q, void *out,
+                            float *lse, float scale, uint32_t *device_error, void *stream);
 
 /* Number of kernel launches the library has enqueued since the cache was allocated. */
 int64_t ripe_launch_count(const ripe_cache_t *c);

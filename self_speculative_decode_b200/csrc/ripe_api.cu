@@ -99,6 +99,7 @@ const char *ripe_strerror(int status) {
         case RIPE_ECAPACITY: return "cache capacity exceeded";
         case RIPE_ESTATE: return "call out of order for the cache state";
         case RIPE_ECUDA: return "CUDA error";
+        case RIPE_ESCRATCH: return "problem exceeds the static scratch of ripe_verify_attn_static";
         default: return "unknown status";
     }
 }

@@ -272,4 +272,21 @@ int launch_export(ripe_cache *c, int n, int layer, void *k_out, void *v_out, uin
                   cudaStream_t s);
 int set_verify_attributes(int d, int N);
 
+// Everything one verify launch needs, for callers that own the buffers and the scratch.
+struct RawVerify {
+    CUtensorMap tmKd, tmVd, tmKw, tmVw;
+    const void *q;
+    void *out;
+    float *lse;
+    const int32_t *T;
+    float *part_o, *part_ml;
+    int32_t *counters;
+    uint32_t *err;
+    PlanArgs plan;
+    int N, kvH, g, Hq, d, layer, grid;
+    float scale;
+};
+int launch_verify_raw(const RawVerify &rv, cudaStream_t s);
+int verify_rows_for(int Mq);  // query rows per partial slot for B * group query rows
+
 }  // namespace ripe

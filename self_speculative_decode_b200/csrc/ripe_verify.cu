@@ -639,6 +639,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 template <int D, int NQT, int WR, int WK, int TG>
 struct Inst {
     using C = VCfg<D, NQT, WR, WK, TG>;
+    static constexpr auto kernel = ripe_verify_kernel<D, NQT, WR, WK, TG>;
     static cudaError_t set_attr(int N) {
         return cudaFuncSetAttribute(ripe_verify_kernel<D, NQT, WR, WK, TG>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for<C>(N));
@@ -648,6 +649,9 @@ struct Inst {
                    smem_bytes_for<C>(c->N), s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
     }
 };
+
+template <class I>
+constexpr auto ripe_verify_kernel_of() { return I::kernel; }
 
 // query-side configuration by the number of query rows per kv head (B * group)
 //   <= 8  : one 8-query tile per warp, 2 tile groups of 4 warps
@@ -685,6 +689,68 @@ static void launch_d(int qc, const ripe_cache *c, int grid, const VerifyArgs &a,
         case 2: I2::launch(c, grid, a, s); break;
         default: I3::launch(c, grid, a, s); break;
     }
+}
+
+// Launch over explicitly given buffers and scratch (the allocation-free entry point).
+template <class I0, class I1, class I2, class I3>
+static cudaError_t launch_raw_d(int qc, const RawVerify &rv, const VerifyArgs &a, cudaStream_t s) {
+    switch (qc) {
+        case 0: return launch_pdl(ripe_verify_kernel_of<I0>(), dim3(rv.grid), dim3(I0::C::THREADS),
+                                  smem_bytes_for<typename I0::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
+        case 1: return launch_pdl(ripe_verify_kernel_of<I1>(), dim3(rv.grid), dim3(I1::C::THREADS),
+                                  smem_bytes_for<typename I1::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
+        case 2: return launch_pdl(ripe_verify_kernel_of<I2>(), dim3(rv.grid), dim3(I2::C::THREADS),
+                                  smem_bytes_for<typename I2::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
+        default: return launch_pdl(ripe_verify_kernel_of<I3>(), dim3(rv.grid), dim3(I3::C::THREADS),
+                                   smem_bytes_for<typename I3::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
+    }
+}
+
+template <class I>
+static cudaError_t set_attr_raw(int N) { return I::set_attr(N); }
+
+template <class I0, class I1, class I2, class I3>
+static cudaError_t set_raw_d(int qc, int N) {
+    switch (qc) {
+        case 0: return set_attr_raw<I0>(N);
+        case 1: return set_attr_raw<I1>(N);
+        case 2: return set_attr_raw<I2>(N);
+        default: return set_attr_raw<I3>(N);
+    }
+}
+
+int verify_rows_for(int Mq) { return 8 << qcfg_of(Mq); }
+
+int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
+    VerifyArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(rv.q);
+    a.out = static_cast<__nv_bfloat16 *>(rv.out);
+    a.lse = rv.lse;
+    a.T = rv.T;
+    a.part_o = rv.part_o;
+    a.part_ml = rv.part_ml;
+    a.counters = rv.counters;
+    a.err = rv.err;
+    a.plan = rv.plan;
+    a.N = rv.N;
+    a.kvH = rv.kvH;
+    a.g = rv.g;
+    a.Hq = rv.Hq;
+    a.B = rv.plan.B;
+    a.R = rv.plan.R;
+    a.layer = rv.layer;
+    a.Mq = rv.plan.B * rv.g;
+    a.min_chunk = RIPE_MIN_CHUNK;
+    a.scale_log2 = rv.scale * 1.4426950408889634f;
+    const int qc = qcfg_of(a.Mq);
+    cudaError_t e;
+    switch (rv.d) {
+        case 64: e = set_raw_d<RIPE_QCFG_LIST(64)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(64)>(qc, rv, a, s); break;
+        case 96: e = set_raw_d<RIPE_QCFG_LIST(96)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(96)>(qc, rv, a, s); break;
+        case 128: e = set_raw_d<RIPE_QCFG_LIST(128)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(128)>(qc, rv, a, s); break;
+        default: return RIPE_EINVAL;
+    }
+    return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,

@@ -22,8 +22,10 @@ EXPORTS = (
     "ripe_cache_alloc", "ripe_cache_free", "ripe_load_prefix", "ripe_append_block",
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
-    "ripe_strerror",
+    "ripe_strerror", "ripe_verify_attn_static",
 )
+RIPE_ESCRATCH = -6
+RIPE_STATIC_SCRATCH_BYTES = 4 << 20
 
 
 class RipeError(RuntimeError):
@@ -37,6 +39,14 @@ class _Stats(ctypes.Structure):
                 ("kv_bytes", ctypes.c_int64), ("scratch_bytes", ctypes.c_int64),
                 ("deep_rows", ctypes.c_int32), ("ring_slots", ctypes.c_int32),
                 ("block_len", ctypes.c_int32), ("lengths_synced", ctypes.c_int32)]
+
+
+class CacheView(ctypes.Structure):
+    """ripe_cache_view: caller-owned cache buffers for ripe_verify_attn_static."""
+    _fields_ = [(name, ctypes.c_int32) for name in
+                ("batch", "layers", "q_heads", "kv_heads", "head_dim", "loops", "window", "max_T",
+                 "max_B", "window_mode", "block_len")] + \
+               [(name, ctypes.c_void_p) for name in ("k_deep", "v_deep", "k_ring", "v_ring", "lengths")]
 
 
 _lib = None
@@ -66,6 +76,7 @@ def lib() -> ctypes.CDLL:
             "ripe_get_device_error": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i),
             "ripe_launch_count": ([vp], i64),
             "ripe_strerror": ([i], ctypes.c_char_p),
+            "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -171,6 +182,14 @@ def ripe_get_device_error(h, stream=None):
     e = ctypes.c_uint32()
     _check(lib().ripe_get_device_error(h, ctypes.byref(e), _stream(stream)), "ripe_get_device_error")
     return e.value
+
+
+def ripe_verify_attn_static(view, layer, r, q, out, lse=None, scale=1.0, device_error=None, stream=None):
+    """Allocation-free verify over caller-owned buffers (see include/ripe.h); pointers are ints."""
+    _check(lib().ripe_verify_attn_static(ctypes.byref(view), layer, r, ctypes.c_void_p(q), ctypes.c_void_p(out),
+                                         ctypes.c_void_p(lse or 0), float(scale),
+                                         ctypes.c_void_p(device_error or 0), _stream(stream)),
+           "ripe_verify_attn_static")
 
 
 def ripe_launch_count(h):
