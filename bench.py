@@ -67,6 +67,36 @@ def verify_bytes(cfg, T_list, r):
     return keys * row + qo
 
 
+def sources_digest():
+    """sha256 over the library's CUDA sources and C header (ties an ncu capture to a kernel version)."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "self_speculative_decode_b200", "csrc", "*.cu*")))
+    files += [os.path.join(ROOT, "include", "ripe.h")]
+    for path in files:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+    return h.hexdigest()
+
+
+def captured_traffic(config):
+    """DRAM bytes per verify launch from the committed ncu summary, if it matches these sources."""
+    path = os.path.join(ROOT, "profiles", "ripe_verify_traffic.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if "=" in line and not line.lstrip().startswith("#"):
+                    k, v = line.split("=", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("sources_sha256") != sources_digest() or f"{config}.bytes_per_launch" not in kv:
+            return None
+        return float(kv[f"{config}.bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -82,7 +112,7 @@ class ClockSampler:
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,utilization.gpu")
 
     def __init__(self, index):
         self.index = index
@@ -94,7 +124,7 @@ class ClockSampler:
         os.close(fd)
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -107,24 +137,29 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons = [], None, set()
+        sm, smax, reasons, loaded = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
+                if len(parts) < 10:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
+                    clk, cmax, util = float(parts[1]), float(parts[2]), float(parts[9])
                 except ValueError:
                     continue
+                smax = cmax
+                if util < 1:       # keep the samples taken while the GPU was busy with the benchmark
+                    continue
+                loaded += 1
+                sm.append(clk)
                 for name, val in zip(names, parts[5:9]):
                     if val.lower() == "active":
                         reasons.add(name)
         os.unlink(self.path)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": loaded, "reasons": sorted(reasons),
+                "window": "every layout's warm-up, timed steps, per-launch and end-to-end timing"}
 
 
 def gpu_id(index):
@@ -232,14 +267,20 @@ def time_region(fn, sync_group):
     return s.elapsed_time(e)  # ms
 
 
-def max_over_ranks(x, dist_on):
+def max_over_ranks(x, dist_on, device="cuda"):
+    """The slowest rank's time: every multi-GPU number is taken as the max over ranks."""
     if not dist_on:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(per_rank_bytes, max_ms, world):
+    """Whole-job GB/s of replicas: every rank moves per_rank_bytes; the job takes the slowest rank's time."""
+    return world * per_rank_bytes / (max_ms * 1e-3) / 1e9
 
 
 def step_bytes(cfg, T_start, acc_rows):
@@ -257,15 +298,10 @@ def bench_layout(cfg, layout, args, seed, device, dist_on, want_extras):
     wl = Workload(cfg, layout, args.warmup + 2 * args.steps + 2, seed, device)
     wl.capture()
     N = cfg["N"]
+    res = {}
     wl.run_steps(0, args.warmup)
     T_start = wl.cache.sync_lengths()
-    res = {}
-    clocks = ClockSampler(gpu_id(torch.cuda.current_device())) if want_extras else None
-    if clocks:
-        clocks.start()
     ms = time_region(lambda: wl.run_steps(args.warmup, args.steps), dist_on)
-    if clocks:
-        res["clocks"] = clocks.stop()
     ms = max_over_ranks(ms, dist_on)
     rows = wl.acc_host[args.warmup:args.warmup + args.steps]
     per_step, T_end = step_bytes(cfg, T_start, rows)
@@ -344,6 +380,20 @@ def e2e_steps(wl, args, dist_on):
                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=ho.numel() * 2)
 
 
+def profile_calls(cfg, args, device):
+    """A few verify calls of one layer of the workload, nothing else: the launch ncu captures."""
+    import torch
+    one = dict(cfg, L=1)
+    wl = Workload(one, "ripe", 1, args.seed, device)
+    for r in range(one["R"]):
+        wl.cache.append_block(0, r, wl.k[0, r], wl.v[0, r])
+    for i in range(args.profile_calls):
+        wl.cache.verify_attn(0, 0, wl.q[0, 0], out=wl.out[0, 0])
+    torch.cuda.synchronize()
+    wl.close()
+    print(json.dumps({"profile_calls": args.profile_calls, "workload": one["workload"] + " (1 layer)"}))
+
+
 # ------------------------------------------------------------------ CPU oracle
 def oracle_sample(cfg, seconds, seed=0, loops=4):
     """Time the CPU oracle on verify calls of layer 0 (loops 0..loops-1 and the deepest),
@@ -416,7 +466,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ripe", choices=["ripe", "reference"])
     ap.add_argument("--config", default="huginn", choices=sorted(CONFIGS))
-    ap.add_argument("--layouts", default="ripe,full,deepest")
+    ap.add_argument("--layouts", default=None,
+                    help="comma list of ripe, full, deepest (default: all three; long_gqa: ripe,deepest)")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="only run this many verify calls of layer 0 (for ncu captures) and exit")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args()
@@ -444,11 +497,21 @@ def main():
     from self_speculative_decode_b200 import ripe
     ripe.lib()
 
+    if args.profile_calls:
+        profile_calls(cfg, args, device)
+        return
+    if args.layouts is None:
+        # the full cache of the long-context config needs R * T * 4 layers (137 GB): not by default
+        args.layouts = "ripe,deepest" if args.config == "long_gqa" else "ripe,full,deepest"
     layouts = [x for x in args.layouts.split(",") if x]
     results = {}
+    clocks = ClockSampler(gpu_id(local))
+    clocks.start()
+    time.sleep(0.3)  # nvidia-smi needs a moment before its first sample
     for lay in layouts:
         results[lay] = bench_layout(cfg, lay, args, args.seed + 1000 * rank, device, dist_on,
                                     want_extras=(lay == layouts[0]))
+    clock_rec = clocks.stop()
     main_l = layouts[0]
     m = results[main_l]
     peak, peak_kind = hbm_peak()
@@ -456,7 +519,7 @@ def main():
     cold = m["verify_cold"]
     achieved = warm["bytes_per_launch"] / (warm["us_per_launch"] * 1e-6) / 1e9
     achieved_cold = cold["bytes_per_launch"] / (cold["us_per_launch"] * 1e-6) / 1e9
-    value = m["gbs"] * world
+    value = job_throughput(m["bytes_per_step"] * args.steps, m["ms_per_step"] * args.steps, world)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
@@ -471,14 +534,14 @@ def main():
         "layouts": {k: {x: v[x] for x in ("ms_per_step", "gbs", "verified_tokens_per_s", "bytes_per_step")}
                     for k, v in results.items()},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                     "frac": achieved / peak, "traffic": captured_traffic(args.config), "peak_kind": peak_kind,
                      "kernel": "ripe_verify_kernel", "launch_us": warm["us_per_launch"],
                      "note": "R*L verify launches back to back as in the step (L2 warm)"},
         "roofline_cold": {"achieved": achieved_cold, "frac": achieved_cold / peak,
                           "launch_us": cold["us_per_launch"], "note": "L2 flushed before each launch"},
         "e2e": m["e2e"],
         "gpu_launches": m["launches_per_step"] * args.steps,
-        "clocks": m.get("clocks"),
+        "clocks": clock_rec,
     }
     if "full" in results and main_l == "ripe":
         line["full_over_ripe_latency"] = results["full"]["ms_per_step"] / m["ms_per_step"]

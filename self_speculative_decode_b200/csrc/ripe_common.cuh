@@ -73,7 +73,7 @@ struct PlanArgs {
 };
 
 struct SeqGeom {
-    int T, D, nd;
+    int T, D, nd, s0;  // s0: ring slot of position D
     int ring_len, ring_first, nr1, nr;
     int dual_len, dual_first, ndl1, ndl;
     int total;
@@ -85,25 +85,30 @@ struct Tile {
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+// ceil(a / box) with the common box of 64 rows as a shift
+__host__ __device__ __forceinline__ int ctiles(int a, int box) {
+    return box == 64 ? (a + 63) >> 6 : cdiv(a, box);
+}
+
 __host__ __device__ __forceinline__ SeqGeom seq_geom(int T, const PlanArgs &a) {
     SeqGeom s;
     s.T = T;
     s.D = T - a.W > 0 ? T - a.W : 0;
-    s.nd = cdiv(s.D, a.deep_box);
-    const int s0 = s.D % a.ring_slots;
+    s.nd = ctiles(s.D, a.deep_box);
+    s.s0 = s.D % a.ring_slots;
     s.ring_len = T + a.B - s.D;
-    s.ring_first = s.ring_len < a.ring_slots - s0 ? s.ring_len : a.ring_slots - s0;
-    s.nr1 = cdiv(s.ring_first, a.ring_box);
-    s.nr = s.nr1 + cdiv(s.ring_len - s.ring_first, a.ring_box);
+    s.ring_first = s.ring_len < a.ring_slots - s.s0 ? s.ring_len : a.ring_slots - s.s0;
+    s.nr1 = ctiles(s.ring_first, a.ring_box);
+    s.nr = s.nr1 + ctiles(s.ring_len - s.ring_first, a.ring_box);
     int dl = 0;
     if (a.mode_eff == 0) {
         const int hi = T < T + a.B - 1 - a.W ? T : T + a.B - 1 - a.W;
         dl = hi - s.D > 0 ? hi - s.D : 0;
     }
     s.dual_len = dl;
-    s.dual_first = dl < a.ring_slots - s0 ? dl : a.ring_slots - s0;
-    s.ndl1 = cdiv(s.dual_first, a.ring_box);
-    s.ndl = s.ndl1 + cdiv(s.dual_len - s.dual_first, a.ring_box);
+    s.dual_first = dl < a.ring_slots - s.s0 ? dl : a.ring_slots - s.s0;
+    s.ndl1 = ctiles(s.dual_first, a.ring_box);
+    s.ndl = s.ndl1 + ctiles(s.dual_len - s.dual_first, a.ring_box);
     s.total = s.nd + s.nr + s.ndl;
     return s;
 }
@@ -129,11 +134,17 @@ __host__ __device__ __forceinline__ Tile tile_at(const SeqGeom &s, int lt, const
         t.kind = kDual; t.plane = a.R - 1;
     }
     int off, seg_end;
-    if (lt < n1) { off = lt * a.ring_box; seg_end = first; }
-    else { off = first + (lt - n1) * a.ring_box; seg_end = len; }
+    if (lt < n1) {  // up to the end of the ring
+        off = lt * a.ring_box;
+        seg_end = first;
+        t.y = s.s0 + off;
+    } else {        // after the wrap, from slot 0
+        off = first + (lt - n1) * a.ring_box;
+        seg_end = len;
+        t.y = off - first;
+    }
     t.t0 = s.D + off;
     t.cnt = (seg_end - off) < a.ring_box ? (seg_end - off) : a.ring_box;
-    t.y = (s.D + off) % a.ring_slots;
     return t;
 }
 
@@ -187,6 +198,11 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
             if (mbar_try_wait(bar, parity)) return true;
         if (global_ns() - t0 > kWaitNs) return false;
     }
+}
+
+// Bring a tensor-map descriptor (a kernel parameter) into the TMA unit's cache ahead of use.
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *m) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
 // 3-D tiled TMA load (no multicast) completing on an mbarrier.
@@ -283,7 +299,7 @@ struct RawVerify {
     int32_t *counters;
     uint32_t *err;
     PlanArgs plan;
-    int N, kvH, g, Hq, d, layer, grid;
+    int N, kvH, g, Hq, d, layer, grid, has_deep;
     float scale;
 };
 int launch_verify_raw(const RawVerify &rv, cudaStream_t s);

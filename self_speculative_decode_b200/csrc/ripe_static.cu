@@ -157,6 +157,7 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.d = d;
     rv.layer = layer;
     rv.grid = grid;
+    rv.has_deep = deep_rows > 0 ? 1 : 0;
     rv.scale = scale;
     const int ls = launch_verify_raw(rv, s);
     if (ls != RIPE_OK) return ls;

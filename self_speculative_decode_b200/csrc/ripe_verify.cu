@@ -45,6 +45,7 @@ struct VerifyArgs {
     uint32_t *err;
     PlanArgs plan;
     int N, kvH, g, Hq, B, R, layer, Mq, min_chunk;
+    int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
     float scale_log2;
 };
 
@@ -53,6 +54,7 @@ constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
 #define RIPE_MIN_CHUNK 4                // at least this many 64-key tiles per CTA
 #endif
 constexpr float kLazyMax = 8.f;     // log2 headroom before the softmax reference moves
+constexpr int kSwitchTiles = 3;     // tiles a CTA may add to its chunk to avoid a mid-stream head switch
 
 // Query-side shapes: NQT 8-query tiles per warp, WR row groups, WK key groups per tile,
 // TG tile groups consuming alternate tiles.
@@ -131,6 +133,14 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const PlanArgs &pa = a.plan;
     const int N = a.N, kvH = a.kvH;
 
+    if (warp == C::NCW && lane == 0) {  // descriptors are parameters: fetch them before the wait
+        tma_prefetch_desc(&tmKw);
+        tma_prefetch_desc(&tmVw);
+        if (a.has_deep) {
+            tma_prefetch_desc(&tmKd);
+            tma_prefetch_desc(&tmVd);
+        }
+    }
     if (tid == 0) {
         sflag[1] = 0;  // abort flag
         sflag[3] = 0;  // pairs this CTA merges at the end (at most its first and last): sflag[4..5]
@@ -171,8 +181,33 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 
     pdl_trigger();  // the next kernel may be scheduled; it waits for this one to finish
     const int total = cum[N];
-    int chunk = cdiv(total, static_cast<int>(gridDim.x));
-    if (chunk < a.min_chunk) chunk = a.min_chunk;
+    if (warp == 0) {
+        // equal tile counts for every (sequence, kv head)?
+        const int tot0 = cum[1] / kvH;
+        bool same = true;
+        for (int b = 0; b < N; b += 32) {
+            const bool ok = (b + lane >= N) || (cum[b + lane + 1] - cum[b + lane] == cum[1]);
+            same = same && __all_sync(0xffffffffu, ok);
+        }
+        if (lane == 0) {
+            int ch = cdiv(total, static_cast<int>(gridDim.x));
+            if (ch < a.min_chunk) ch = a.min_chunk;
+            if (same) {
+                // cut at (sequence, kv head) boundaries when that costs at most kSwitchTiles
+                // tiles per CTA: a CTA then never switches to another head mid-stream
+                if (ch < tot0) {
+                    const int ca = cdiv(tot0, tot0 / ch);
+                    if (ca <= ch + kSwitchTiles) ch = ca;
+                } else {
+                    const int ca = cdiv(ch, tot0) * tot0;
+                    if (ca <= ch + kSwitchTiles) ch = ca;
+                }
+            }
+            sflag[6] = ch;
+        }
+    }
+    __syncthreads();
+    const int chunk = sflag[6];
     const int g_begin = blockIdx.x * chunk;
     const int g_end = min(total, g_begin + chunk);
     if (g_begin >= g_end) return;
@@ -658,8 +693,12 @@ constexpr auto ripe_verify_kernel_of() { return I::kernel; }
 //   <= 16 : two 8-query tiles per warp, 2 tile groups of 4 warps
 //   <= 32 : two row groups x 4 key groups
 //   <= 64 : four row groups x 2 key groups (32 keys per warp per tile)
+#ifndef RIPE_Q8_WK
+#define RIPE_Q8_WK 4
+#define RIPE_Q8_TG 2
+#endif
 #define RIPE_QCFG_LIST(D)                                                          \
-    Inst<D, 1, 1, 4, 2>, Inst<D, 2, 1, 4, 2>, Inst<D, 2, 2, 4, 1>, Inst<D, 2, 4, 2, 1>
+    Inst<D, 1, 1, RIPE_Q8_WK, RIPE_Q8_TG>, Inst<D, 2, 1, 4, 2>, Inst<D, 2, 2, 4, 1>, Inst<D, 2, 4, 2, 1>
 
 static int qcfg_of(int Mq) { return Mq <= 8 ? 0 : Mq <= 16 ? 1 : Mq <= 32 ? 2 : 3; }
 
@@ -741,6 +780,7 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.layer = rv.layer;
     a.Mq = rv.plan.B * rv.g;
     a.min_chunk = RIPE_MIN_CHUNK;
+    a.has_deep = rv.has_deep;
     a.scale_log2 = rv.scale * 1.4426950408889634f;
     const int qc = qcfg_of(a.Mq);
     cudaError_t e;
@@ -782,6 +822,7 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
     a.layer = layer;
     a.Mq = c->B_cur * c->g;
     a.min_chunk = RIPE_MIN_CHUNK;  // bounds the number of partials of one (sequence, kv head)
+    a.has_deep = c->deep_rows > 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
     const int qc = qcfg_of(a.Mq);
 
