@@ -613,9 +613,10 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 const float p3 = (r1 == -INFINITY) ? 0.f : exp2f(x[sb][nq][3] - r1);
                 const __nv_bfloat162 lo = __floats2bfloat162_rn(p0, p1);
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(p2, p3);
-                const float2 flo = __bfloat1622float2(lo), fhi = __bfloat1622float2(hi);
-                l_run[nq][0] += flo.x + fhi.x;
-                l_run[nq][1] += flo.y + fhi.y;
+                // the normaliser sums the fp32 probabilities (the lse stays fp32-accurate);
+                // only the P V product sees them rounded to bf16
+                l_run[nq][0] += p0 + p2;
+                l_run[nq][1] += p1 + p3;
                 pb[nq][0] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&lo));
                 pb[nq][1] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&hi));
             }

@@ -16,8 +16,10 @@ from self_speculative_decode_b200.synth import PlaneSource
 # bf16 inputs, fp32 accumulation, bf16 output: the tolerance the benchmark spec fixes for the verify output
 MAX_ABS = 2e-2
 REL_L2 = 5e-3
-# the log-sum-exp is returned in fp32 (no bf16 rounding): its error is the fp32 softmax sum's
-LSE_ABS = 2e-3
+# the log-sum-exp is returned in fp32 from an fp32 sum of up to ~33K exponentials: its error is
+# bounded by the sum's rounding (< 33K * 2^-24 relative) plus the approximate exp2 / log2 (~2^-22
+# relative each), well under 1e-3 in absolute terms for logits of moderate size
+LSE_ABS = 1e-3
 
 
 def bits_to_dev(bits: np.ndarray, device) -> torch.Tensor:
@@ -56,6 +58,18 @@ def check_lse(gpu_lse: torch.Tensor, ref: np.ndarray):
     err = np.abs(got - ref).max()
     assert err <= LSE_ABS, f"lse: max abs error {err:.3e}"
     return float(err)
+
+
+def assert_same_result(a: torch.Tensor, b: torch.Tensor, what: str = ""):
+    """Two GPU results of the same attention with a different split of the key range.
+
+    Each is within MAX_ABS / REL_L2 of the exact value (the parity tolerance: bf16 P and
+    output rounding, fp32 sums), so by the triangle inequality they are within twice that
+    of each other."""
+    a, b = a.double(), b.double()
+    err = (a - b).abs().max().item()
+    rel = (torch.linalg.vector_norm(a - b) / torch.clamp(torch.linalg.vector_norm(a), min=1e-30)).item()
+    assert err <= 2 * MAX_ABS and rel <= 2 * REL_L2, f"{what}: max abs {err:.3e}, relative L2 {rel:.3e}"
 
 
 class Case:
