@@ -97,6 +97,25 @@ def captured_traffic(config):
         return None
 
 
+def wave_loops(cfg):
+    """A diagonal wavefront: block position j at loop R-1-4j (older positions deeper)."""
+    return [max(0, cfg["R"] - 1 - 4 * j) for j in range(cfg["B"])]
+
+
+def wave_bytes(cfg, T_list, W):
+    """Algorithmic bytes of one wavefront call: the deepest region once, the window ring once
+    per distinct loop, the dual window keys, queries and outputs."""
+    loops = wave_loops(cfg)
+    nl = len(set(loops))
+    row = 4 * cfg["kvH"] * cfg["d"]
+    keys = 0
+    for T in T_list:
+        D = max(0, T - W)
+        dual = max(0, min(T, T + cfg["B"] - 1 - W) - D)
+        keys += D + nl * (T + cfg["B"] - D) + dual
+    return keys * row + 2 * cfg["N"] * cfg["B"] * cfg["Hq"] * cfg["d"] * 2
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -343,10 +362,34 @@ def bench_layout(cfg, layout, args, seed, device, dist_on, want_extras):
                                   bytes_per_launch=sum(x for _, _, x in evs) / len(evs))
         del flush
         res["e2e"] = e2e_steps(wl, args, dist_on)
+    if layout in ("ripe", "full"):
+        res["wave"] = wave_timing(wl, args, dist_on)
     wl.close()
     del wl
     torch.cuda.empty_cache()
     return res
+
+
+def wave_timing(wl, args, dist_on):
+    """One wavefront call per layer (block positions at different loops), as a CUDA graph."""
+    import torch
+    cfg, c = wl.cfg, wl.cache
+    if c.stats()["block_len"] == 0:
+        for r in range(cfg["R"]):
+            for layer in range(cfg["L"]):
+                c.append_block(layer, r, wl.k[layer, r], wl.v[layer, r])
+    loops = wave_loops(cfg)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for layer in range(cfg["L"]):
+            c.verify_attn_wave(layer, loops, wl.q[layer, 0], out=wl.out[layer, 0])
+    reps = max(3, args.steps)
+    g.replay()
+    ms = max_over_ranks(time_region(lambda: [g.replay() for _ in range(reps)], dist_on), dist_on)
+    T_now = c.sync_lengths()
+    us = ms * 1e3 / (reps * cfg["L"])
+    nbytes = wave_bytes(cfg, T_now, wl.W)
+    return dict(us_per_call=us, bytes_per_call=nbytes, gbs=nbytes / (us * 1e-6) / 1e9, loops=loops)
 
 
 def e2e_steps(wl, args, dist_on):
@@ -545,6 +588,14 @@ def main():
     }
     if "full" in results and main_l == "ripe":
         line["full_over_ripe_latency"] = results["full"]["ms_per_step"] / m["ms_per_step"]
+        wr, wf = results["ripe"]["wave"], results["full"]["wave"]
+        line["wavefront"] = {
+            "loops": wr["loops"], "ripe_us": wr["us_per_call"], "full_us": wf["us_per_call"],
+            "latency_ratio_full_over_ripe": wf["us_per_call"] / wr["us_per_call"],
+            "bytes_ratio_full_over_ripe": wf["bytes_per_call"] / wr["bytes_per_call"],
+            "ripe_gbs": wr["gbs"], "full_gbs": wf["gbs"],
+            "note": "one call per layer verifies every block position at its own loop; the deepest "
+                    "region is read once for all loops, the window once per loop"}
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         gbs, calls, sec, threads = oracle_sample(cfg, args.cpu_seconds)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",

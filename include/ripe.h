@@ -150,6 +150,21 @@ int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out
                      float scale, void *stream);
 
 /*
+ * Verification attention with a loop per block position: block position j is evaluated
+ * exactly as ripe_verify_attn(.., loop_of_position[j], ..) would evaluate it.  This is the
+ * shape of a wavefront schedule, where one batched pass of the looped block holds positions
+ * at different depths (WaveFront write-up, sections on drafting and checking in one pass and on
+ * the long-context bottleneck: positions at different depths read different KV regions).
+ * The deepest-plane region is read once for all positions; the window ring once per distinct
+ * loop.  With RIPE this reads T + n_loops * (W + B) key rows per (sequence, kv head), where a
+ * full cache reads n_loops * (T + B).
+ *   loop_of_position  host int32[B], each 0 .. R-1 with that plane of the block appended
+ *   q, out, lse, scale as for ripe_verify_attn
+ */
+int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q,
+                          void *out, float *lse, float scale, void *stream);
+
+/*
  * Accept a prefix of the draft block of every sequence and roll back the rest
  * (WaveFront write-up, draft-then-verify): accepted_len[n] in 0 .. B positions of the block
  * become committed, T_n += accepted_len[n]; the other block positions are discarded.

@@ -19,6 +19,9 @@ Contents
                        rollback and window eviction.
   * ``memory_fraction`` stored fraction of the full cache, counted from the state
                        machine.
+  * ``verify_wave``    a loop per block position: each position evaluated as the
+                       single-loop verification at its own loop (definition by
+                       composition).
 Every function here is pinned by ``tests/test_oracle_*.py``; none is "parity
 unpinned".
 """
@@ -272,6 +275,25 @@ class OracleCache:
         Kr, Vr, Kl, Vl, _ = self.verify_inputs(layer, r)
         return verify(self.T, self.B, r, self.R, self.W, g, Kr, Vr, Kl, Vl,
                       bf16_to_f64(q_bits), scale, self.mode)
+
+
+def verify_wave(cache, layer, loop_of_position, q_bits, g, scale=1.0):
+    """Verification with a loop per block position (several depths in one call, as in a
+    wavefront schedule): block position j is evaluated exactly as a single-loop verification
+    at loop loop_of_position[j] would evaluate it.  Returns (out, lse) in fp64."""
+    loops = [int(x) for x in loop_of_position]
+    if len(loops) != cache.B:
+        raise ValueError("one loop per block position")
+    out = lse = None
+    for r in sorted(set(loops)):
+        o, l = cache.verify(layer, r, q_bits, g, scale)
+        if out is None:
+            out, lse = np.zeros_like(o), np.zeros_like(l)
+        for j, rj in enumerate(loops):
+            if rj == r:
+                out[:, j] = o[:, j]
+                lse[:, j] = l[:, j]
+    return out, lse
 
 
 def memory_fraction(T, W, R, recurrent_layers=1, other_layers=0, B=1):

@@ -234,6 +234,20 @@ int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out
     return launch_verify(c, layer, r, q, out, lse, scale, static_cast<cudaStream_t>(stream));
 }
 
+int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
+                          float *lse, float scale, void *stream) {
+    if (!c || !loop_of_position || !q || !out || layer < 0 || layer >= c->L) return RIPE_EINVAL;
+    if (c->B_cur == 0) return RIPE_ESTATE;
+    for (int j = 0; j < c->B_cur; ++j) {
+        const int r = loop_of_position[j];
+        if (r < 0 || r >= c->R) return RIPE_EINVAL;
+        if (!c->appended[static_cast<size_t>(layer) * c->R + r]) return RIPE_ESTATE;
+    }
+    DeviceGuard g(c->device);
+    if (!g.ok) return RIPE_ECUDA;
+    return launch_verify_wave(c, layer, loop_of_position, q, out, lse, scale, static_cast<cudaStream_t>(stream));
+}
+
 int ripe_commit(ripe_cache_t *c, const int32_t *accepted_len, void *stream) {
     if (!c || !accepted_len) return RIPE_EINVAL;
     if (c->B_cur == 0 || !all_appended(c)) return RIPE_ESTATE;

@@ -62,14 +62,18 @@ namespace ripe {
 // ---------------------------------------------------------------- tile plan
 // The keys of one (sequence, kv head) at loop r form a list of tiles:
 //   DEEP  the deepest-plane region, positions [0, D), D = max(0, T - W)
-//   RING  positions [D, T + B) at plane r from the window ring (window + draft block)
+//   RING  positions [D, T + B) at plane r from the window ring (window + draft block), once
+//         for every distinct loop r of the call (queries of other loops do not see it)
 //   DUAL  positions [D, min(T, T + B - 1 - W)) at plane R-1 from the ring: window keys
 //         that are older than W for the later queries of the block (query-relative rule)
 // Ring ranges are cut where the ring wraps, so every tile is one box of consecutive slots.
 enum TileKind { kDeep = 0, kRing = 1, kDual = 2 };
 
 struct PlanArgs {
-    int W, B, R, r, ring_slots, deep_box, ring_box, mode_eff;
+    int W, B, R, ring_slots, deep_box, ring_box, mode_eff;
+    int nloops;                      // distinct loops of this call (1 for a single-loop verify)
+    uint8_t loop[kMaxQueryRows];     // those loops; the ring is read once per loop
+    uint8_t jloop[kMaxQueryRows];    // loop of each block position j
 };
 
 struct SeqGeom {
@@ -109,7 +113,7 @@ __host__ __device__ __forceinline__ SeqGeom seq_geom(int T, const PlanArgs &a) {
     s.dual_first = dl < a.ring_slots - s.s0 ? dl : a.ring_slots - s.s0;
     s.ndl1 = ctiles(s.dual_first, a.ring_box);
     s.ndl = s.ndl1 + ctiles(s.dual_len - s.dual_first, a.ring_box);
-    s.total = s.nd + s.nr + s.ndl;
+    s.total = s.nd + a.nloops * s.nr + s.ndl;
     return s;
 }
 
@@ -125,11 +129,13 @@ __host__ __device__ __forceinline__ Tile tile_at(const SeqGeom &s, int lt, const
     }
     lt -= s.nd;
     int len, first, n1;
-    if (lt < s.nr) {
+    if (lt < a.nloops * s.nr) {
+        int k = 0;
+        while (lt >= s.nr) { lt -= s.nr; ++k; }
         len = s.ring_len; first = s.ring_first; n1 = s.nr1;
-        t.kind = kRing; t.plane = a.r;
+        t.kind = kRing; t.plane = a.loop[k];
     } else {
-        lt -= s.nr;
+        lt -= a.nloops * s.nr;
         len = s.dual_len; first = s.dual_first; n1 = s.ndl1;
         t.kind = kDual; t.plane = a.R - 1;
     }
@@ -279,6 +285,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // ---------------------------------------------------------------- launchers (defined per .cu)
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
                   float scale, cudaStream_t s);
+int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q,
+                       void *out, float *lse, float scale, cudaStream_t s);
 int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const void *v,
                   cudaStream_t s);
 int launch_commit(ripe_cache *c, const int32_t *acc_host, const int32_t *acc_dev, cudaStream_t s);

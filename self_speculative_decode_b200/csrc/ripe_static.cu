@@ -145,7 +145,9 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.plan.W = W;
     rv.plan.B = v->block_len;
     rv.plan.R = R;
-    rv.plan.r = r;
+    rv.plan.nloops = 1;
+    rv.plan.loop[0] = static_cast<uint8_t>(r);
+    for (int j = 0; j < kMaxQueryRows; ++j) rv.plan.jloop[j] = static_cast<uint8_t>(r);
     rv.plan.ring_slots = S;
     rv.plan.deep_box = deep_box;
     rv.plan.ring_box = ring_box;

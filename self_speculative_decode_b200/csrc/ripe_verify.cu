@@ -82,7 +82,7 @@ struct VCfg {
 };
 
 struct TileDesc {
-    int pair, n, kh, T, kind, t0, cnt, pad;
+    int pair, n, kh, T, kind, t0, cnt, plane;
 };
 
 template <class C>
@@ -243,7 +243,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                                    : (((a.layer * N + n) * a.R + t.plane) * kvH + kh);
                 TileDesc &dsc = sdesc[s];
                 dsc.pair = n * kvH + kh; dsc.n = n; dsc.kh = kh; dsc.T = sg.T;
-                dsc.kind = t.kind; dsc.t0 = t.t0; dsc.cnt = t.cnt;
+                dsc.kind = t.kind; dsc.t0 = t.t0; dsc.cnt = t.cnt; dsc.plane = t.plane;
                 const uint32_t fb = full0 + 8 * s;
                 mbar_expect_tx(fb, 2 * C::NBOX * rows * 64);
                 const uint32_t kdst = stage0 + s * C::STAGE_BYTES;
@@ -291,7 +291,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const int nct = C::NCW * 32;
 
     // query columns held by this thread: q = NQ*rg + 8*nq + 2*c4 + e  (e = 0, 1)
-    int jq[NQT][2];
+    int jq[NQT][2], lq[NQT][2];  // block position and loop of each query column held
     bool qvalid[NQT][2];
 #pragma unroll
     for (int nq = 0; nq < NQT; ++nq)
@@ -300,6 +300,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             const int i = C::NQ * rg + 8 * nq + 2 * c4 + e;
             qvalid[nq][e] = i < a.Mq;
             jq[nq][e] = qvalid[nq][e] ? i / a.g : a.B - 1;
+            lq[nq][e] = qvalid[nq][e] ? pa.jloop[jq[nq][e]] : -1;
         }
     // ldmatrix lane geometry (64-byte swizzle: 16-byte chunk ^= (row >> 1) & 3)
     const int mi = lane >> 3, r8 = lane & 7;
@@ -557,8 +558,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                         const int tpos = dsc.t0 + kk;
                         const int pq = dsc.T + jq[nq][e & 1];
                         bool vis = act[sb] && kk < dsc.cnt;
-                        if (dsc.kind == kRing)
-                            vis = vis && tpos <= pq && (pa.mode_eff != 0 || tpos >= dsc.T || tpos >= pq - pa.W);
+                        if (dsc.kind == kRing)  // the ring at plane r serves only the queries of loop r
+                            vis = vis && lq[nq][e & 1] == dsc.plane && tpos <= pq &&
+                                  (pa.mode_eff != 0 || tpos >= dsc.T || tpos >= pq - pa.W);
                         else if (dsc.kind == kDual)
                             vis = vis && tpos < pq - pa.W;
                         v = vis ? v : -INFINITY;
@@ -794,6 +796,8 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 
+static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s);
+
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,
                   cudaStream_t s) {
     VerifyArgs a;
@@ -808,12 +812,47 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
     a.plan.W = c->W;
     a.plan.B = c->B_cur;
     a.plan.R = c->R;
-    a.plan.r = r;
     a.plan.ring_slots = c->ring_slots;
     a.plan.deep_box = c->deep_box;
     a.plan.ring_box = c->ring_box;
     // at the deepest loop every key reads plane R-1, so the window rule changes nothing
     a.plan.mode_eff = (c->mode == RIPE_WINDOW_CACHE_RELATIVE || r == c->R - 1) ? 1 : 0;
+    a.plan.nloops = 1;
+    a.plan.loop[0] = static_cast<uint8_t>(r);
+    for (int j = 0; j < kMaxQueryRows; ++j) a.plan.jloop[j] = static_cast<uint8_t>(r);
+    return launch_cache_args(c, layer, a, scale, s);
+}
+
+// Several loops in one call: block position j is verified at loop loop_of_position[j].
+int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
+                       float *lse, float scale, cudaStream_t s) {
+    VerifyArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.plan.W = c->W;
+    a.plan.B = c->B_cur;
+    a.plan.R = c->R;
+    a.plan.ring_slots = c->ring_slots;
+    a.plan.deep_box = c->deep_box;
+    a.plan.ring_box = c->ring_box;
+    a.plan.mode_eff = c->mode == RIPE_WINDOW_CACHE_RELATIVE ? 1 : 0;
+    bool used[kMaxLoops] = {false};
+    for (int j = 0; j < c->B_cur; ++j) used[loop_of_position[j]] = true;
+    a.plan.nloops = 0;
+    for (int r = 0; r < c->R; ++r)
+        if (used[r]) a.plan.loop[a.plan.nloops++] = static_cast<uint8_t>(r);
+    for (int j = 0; j < kMaxQueryRows; ++j)
+        a.plan.jloop[j] = static_cast<uint8_t>(j < c->B_cur ? loop_of_position[j] : loop_of_position[0]);
+    return launch_cache_args(c, layer, a, scale, s);
+}
+
+static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s) {
+    a.T = c->T_dev;
+    a.part_o = c->part_o;
+    a.part_ml = c->part_ml;
+    a.counters = c->counters;
+    a.err = c->err_dev;
     a.N = c->N;
     a.kvH = c->kvH;
     a.g = c->g;

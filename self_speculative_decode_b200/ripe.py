@@ -22,7 +22,7 @@ EXPORTS = (
     "ripe_cache_alloc", "ripe_cache_free", "ripe_load_prefix", "ripe_append_block",
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
-    "ripe_strerror", "ripe_verify_attn_static",
+    "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
             "ripe_launch_count": ([vp], i64),
             "ripe_strerror": ([i], ctypes.c_char_p),
             "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
+            "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -151,6 +152,12 @@ def ripe_verify_attn(h, layer, r, q, out, lse=None, scale=1.0, stream=None):
     _check(lib().ripe_verify_attn(h, layer, r, ctypes.c_void_p(q), ctypes.c_void_p(out),
                                   ctypes.c_void_p(lse or 0), float(scale), _stream(stream)),
            "ripe_verify_attn")
+
+
+def ripe_verify_attn_wave(h, layer, loop_of_position, q, out, lse=None, scale=1.0, stream=None):
+    _check(lib().ripe_verify_attn_wave(h, layer, _ints(loop_of_position, len(loop_of_position)),
+                                       ctypes.c_void_p(q), ctypes.c_void_p(out), ctypes.c_void_p(lse or 0),
+                                       float(scale), _stream(stream)), "ripe_verify_attn_wave")
 
 
 def ripe_commit(h, accepted_len, stream=None):
@@ -251,6 +258,19 @@ class RipeCache:
         op = _dev(out, torch.bfloat16, shape, "out").value
         lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
         ripe_verify_attn(self.handle, layer, r, qp, op, lp, scale, stream)
+        return out
+
+    def verify_attn_wave(self, layer, loop_of_position, q, out=None, lse=None, scale=1.0, stream=None):
+        """Block position j verified at loop loop_of_position[j] (one pass over the deepest plane)."""
+        import torch
+        B = q.shape[1]
+        shape = (self.N, B, self.Hq, self.d)
+        qp = _dev(q, torch.bfloat16, shape, "q").value
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+        op = _dev(out, torch.bfloat16, shape, "out").value
+        lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
+        ripe_verify_attn_wave(self.handle, layer, list(loop_of_position), qp, op, lp, scale, stream)
         return out
 
     def commit(self, accepted_len, stream=None):

@@ -158,6 +158,18 @@ class Case:
         gl = lse.index_select(0, idx_n).index_select(2, idx_h) if with_lse else None
         return go, gl, ro, rl
 
+    def check_wave(self, layer, loops, scale=1.0):
+        """A loop per block position, against the oracle's per-position composition."""
+        qd, qh = self.queries(layer, 0, step=7)
+        lse = torch.empty((self.N, self.B, self.Hq), dtype=torch.float32, device=self.device)
+        out = self.gpu.verify_attn_wave(layer, loops, qd, lse=lse, scale=scale)
+        ro, rl = orc.verify_wave(self.orc, layer, loops, qh, self.g, scale)
+        idx_n = torch.tensor(self.oseq, device=self.device)
+        idx_h = torch.tensor(self.oheads, device=self.device)
+        e = check_close(out.index_select(0, idx_n).index_select(2, idx_h), ro, f"layer {layer} loops {loops}")
+        check_lse(lse.index_select(0, idx_n).index_select(2, idx_h), rl)
+        return e
+
     def check(self, layer, r, scale=1.0):
         go, gl, ro, rl = self.run(layer, r, scale)
         e = check_close(go, ro, f"layer {layer} loop {r}")

@@ -274,3 +274,24 @@ def test_rollback_discards_rejected_positions_and_evicts():
         for r in range(R):
             c.append(0, r, blk(1, 2), blk(1, 2))
         c.commit([3])              # more than the block length
+
+
+# ---------------------------------------------------------------- loop per position (wavefront)
+def test_wave_rows_match_the_brute_force_at_each_rows_loop():
+    """Each block position evaluated at its own loop equals the independent brute-force
+    formulation run at that loop, row by row (a diagonal wave: older positions deeper)."""
+    N, kvH, g, d, R, W, T, B = 1, 2, 2, 8, 6, 3, 20, 5
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W, T, B, seed=13, independent=True)
+    loops = [5, 4, 2, 1, 0]
+    q = src.queries(0, B, kvH * g)
+    out, lse = orc.verify_wave(c, 0, loops, q, g, 1.1)
+    Kall = np.stack([_f64(PK[pl][0]) for pl in range(R)])
+    Vall = np.stack([_f64(PV[pl][0]) for pl in range(R)])
+    for j, r in enumerate(loops):
+        bo, bl = orc.brute_verify(Kall, Vall, T, B, r, W, g, _f64(q[0]), 1.1)
+        assert np.abs(out[0, j] - bo[j]).max() < 1e-12
+        assert np.abs(lse[0, j] - bl[j]).max() < 1e-12
+    # a single loop for every position is the ordinary verification
+    o1, _ = orc.verify_wave(c, 0, [3] * B, q, g)
+    o2, _ = c.verify(0, 3, q, g)
+    assert np.array_equal(o1, o2)
