@@ -233,9 +233,11 @@ class Workload:
         c, cfg = self.cache, self.cfg
         for r in range(cfg["R"]):
             for layer in range(cfg["L"]):
-                if not verify_only:
-                    c.append_block(layer, r, self.k[layer, r], self.v[layer, r])
-                c.verify_attn(layer, r, self.q[layer, r], out=self.out[layer, r])
+                if verify_only:
+                    c.verify_attn(layer, r, self.q[layer, r], out=self.out[layer, r])
+                else:  # append plane r of the block and verify at loop r: one launch
+                    c.append_verify(layer, r, self.k[layer, r], self.v[layer, r], self.q[layer, r],
+                                    out=self.out[layer, r])
 
     def capture(self):
         import torch
@@ -568,7 +570,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg["workload"], "layout": main_l,
-                   "step": "R*L x (append plane r + verify at loop r) + commit/evict, CUDA graph",
+                   "step": "R*L x fused (append plane r + verify at loop r) + commit/evict, CUDA graph",
                    "T_range": m["T_range"], "l2": "inputs larger than L2 (every step reads the whole cache)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": 100.0 * m["gbs"] / peak,

@@ -150,6 +150,15 @@ int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out
                      float scale, void *stream);
 
 /*
+ * ripe_append_block(c, layer, r, B, k, v) followed by ripe_verify_attn(c, layer, r, q, ...) in
+ * one launch: plane r of the draft block is written into the window ring by the verify kernel
+ * itself, just before the one tile of this launch that reads those rows.  Arguments, layouts,
+ * results and errors are those of the two calls; the result is identical.
+ */
+int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, const void *v,
+                       const void *q, void *out, float *lse, float scale, void *stream);
+
+/*
  * Verification attention with a loop per block position: block position j is evaluated
  * exactly as ripe_verify_attn(.., loop_of_position[j], ..) would evaluate it.  This is the
  * shape of a wavefront schedule, where one batched pass of the looped block holds positions

@@ -234,6 +234,28 @@ int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out
     return launch_verify(c, layer, r, q, out, lse, scale, static_cast<cudaStream_t>(stream));
 }
 
+int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, const void *v, const void *q,
+                       void *out, float *lse, float scale, void *stream) {
+    if (!c || !k || !v || !q || !out || layer < 0 || layer >= c->L || r < 0 || r >= c->R || B < 1 ||
+        B > c->max_B)
+        return RIPE_EINVAL;
+    if (c->B_cur != 0 && B != c->B_cur) return RIPE_EINVAL;
+    for (int n = 0; n < c->N; ++n)
+        if (c->T[n] + B > c->max_T) return RIPE_ECAPACITY;
+    DeviceGuard g(c->device);
+    if (!g.ok) return RIPE_ECUDA;
+    const int prev_B = c->B_cur;
+    c->B_cur = B;  // the kernel plans the block's tiles with this length
+    const int st = launch_verify(c, layer, r, q, out, lse, scale, static_cast<cudaStream_t>(stream), k, v);
+    if (st != RIPE_OK) {
+        c->B_cur = prev_B;
+        return st;
+    }
+    c->appended[static_cast<size_t>(layer) * c->R + r] = 1;
+    c->prefix_set = true;
+    return RIPE_OK;
+}
+
 int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                           float *lse, float scale, void *stream) {
     if (!c || !loop_of_position || !q || !out || layer < 0 || layer >= c->L) return RIPE_EINVAL;

@@ -284,7 +284,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 // ---------------------------------------------------------------- launchers (defined per .cu)
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
-                  float scale, cudaStream_t s);
+                  float scale, cudaStream_t s, const void *blk_k = nullptr, const void *blk_v = nullptr);
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q,
                        void *out, float *lse, float scale, cudaStream_t s);
 int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const void *v,

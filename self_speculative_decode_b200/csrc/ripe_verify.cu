@@ -47,9 +47,21 @@ struct VerifyArgs {
     int N, kvH, g, Hq, B, R, layer, Mq, min_chunk;
     int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
     float scale_log2;
+    // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
+    const uint4 *blk_k, *blk_v;
+    uint4 *ring_k, *ring_v;
+    int max_T;
 };
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
+#ifndef RIPE_MAX_STAGES
+#define RIPE_MAX_STAGES 8               // TMA pipeline depth cap (shared memory sets the rest)
+#endif
+#ifndef RIPE_MAX_STAGES_WIDE
+// head_dim 128 with a single tile group (16-32-query rows per kv head, GQA): 3 stages of 32 KB
+// measured faster than 2 or 4 on B200 (long-context GQA verify: 204 vs 230 / 218 us)
+#define RIPE_MAX_STAGES_WIDE 3
+#endif
 #ifndef RIPE_MIN_CHUNK
 #define RIPE_MIN_CHUNK 4                // at least this many 64-key tiles per CTA
 #endif
@@ -73,12 +85,17 @@ struct VCfg {
     static constexpr int MLF = NCW * NQ * 2 + ROWS * (TG * WK + 2);
     static constexpr int MISC = 1024 /*align*/ + 1024 /*bars, descriptors, flags*/;
     static constexpr int AVAIL = kSmemLimit - MISC - 4 * (MERGE_FLOATS + MLF) - 4 * (2 * kMaxBatch + 2);
-    static constexpr int NS_RAW = AVAIL / STAGE_BYTES > 8 ? 8 : AVAIL / STAGE_BYTES;
+    static constexpr int CAP = (D == 128 && TG == 1) ? RIPE_MAX_STAGES_WIDE : RIPE_MAX_STAGES;
+    static constexpr int NS_RAW = AVAIL / STAGE_BYTES > CAP ? CAP : AVAIL / STAGE_BYTES;
     static constexpr int NS = NS_RAW - NS_RAW % TG;
     static_assert(NS >= 2, "not enough shared memory for the pipeline");
     static constexpr int SMEM_FIXED = MISC + NS * STAGE_BYTES + 4 * (MERGE_FLOATS + MLF);
-    // the end-of-CTA merge keeps m and l of up to 256 partials per query row in the stage buffers
-    static_assert(NS * STAGE_BYTES >= 2 * 256 * ROWS * 4, "stage buffers too small for the merge");
+    // the end-of-CTA merge keeps m and l of every partial of a query row in the stage buffers:
+    // at most MAX_PARTS partials, so at most MAX_PARTS CTAs (enough for a 148-SM B200)
+    static constexpr int MAX_PARTS = (NS * STAGE_BYTES) / (2 * ROWS * 4) < 256 ? (NS * STAGE_BYTES) / (2 * ROWS * 4) : 256;
+#ifndef RIPE_ALLOW_SMALL_GRID
+    static_assert(MAX_PARTS >= 148, "stage buffers too small for the end-of-CTA merge");
+#endif
 };
 
 struct TileDesc {
@@ -106,6 +123,44 @@ __device__ __forceinline__ int pair_of(const int *cum, int N, int kvH, int gt) {
     return n * kvH + (gt - cum[n]) / tot;
 }
 
+// Fused append: the rows of the draft block (positions >= T) inside this CTA's ring tiles are
+// copied from the caller's block K/V [N][B][kvH][d] into ring plane r.  No other tile of the
+// launch reads those slots.  Kept out of line: it runs once per CTA, away from the tile loop.
+template <int D>
+__device__ __noinline__ void fused_block_copy(const VerifyArgs &a, const int *cum, const int *Ts, int g_begin,
+                                              int g_end, int tid, int nthreads) {
+    const PlanArgs &pa = a.plan;
+    const int N = a.N, kvH = a.kvH;
+    const int p_first = pair_of(cum, N, kvH, g_begin), p_last = pair_of(cum, N, kvH, g_end - 1);
+    const int d8 = D / 8;
+    for (int p = p_first; p <= p_last; ++p) {
+        const int n = p / kvH, kh = p - (p / kvH) * kvH;
+        const SeqGeom sg = seq_geom(Ts[n], pa);
+        if (sg.T + a.B > a.max_T) {
+            if (tid == 0) atomicOr(a.err, RIPE_DEVERR_CAPACITY);
+            continue;
+        }
+        const int start = cum[n] + kh * sg.total;
+        for (int lt = sg.nd; lt < sg.nd + sg.nr; ++lt) {
+            const int gt = start + lt;
+            if (gt < g_begin || gt >= g_end) continue;
+            const Tile t = tile_at(sg, lt, pa);
+            if (t.t0 + t.cnt <= sg.T) continue;
+            const int r0 = t.t0 > sg.T ? t.t0 : sg.T;
+            const int rows = t.t0 + t.cnt - r0;
+            for (int e = tid; e < rows * d8; e += nthreads) {
+                const int row = e / d8, c8 = e - (e / d8) * d8;
+                const int tpos = r0 + row;
+                const size_t src = ((static_cast<size_t>(n) * a.B + (tpos - sg.T)) * kvH + kh) * d8 + c8;
+                const size_t dst = ((((static_cast<size_t>(a.layer) * N + n) * a.R + t.plane) * kvH + kh) *
+                                        pa.ring_slots + (t.y + (tpos - t.t0))) * d8 + c8;
+                a.ring_k[dst] = a.blk_k[src];
+                a.ring_v[dst] = a.blk_v[src];
+            }
+        }
+    }
+}
+
 template <int D, int NQT, int WR, int WK, int TG>
 __global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS, 1)
 ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_constant__ CUtensorMap tmVd,
@@ -121,8 +176,8 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     float *mml = mo + C::MERGE_FLOATS;                                   // [NCW][NQ][2]
     float *wq = mml + C::NCW * C::NQ * 2;                                // [ROWS][TG*WK] weights
     float *fin = wq + C::ROWS * TG * WK;                                 // [ROWS][2] final M, L
-    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);         // full[NS], empty[NS]
-    TileDesc *sdesc = reinterpret_cast<TileDesc *>(bars + 2 * NS);       // [NS]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);         // full[NS], empty[NS], block
+    TileDesc *sdesc = reinterpret_cast<TileDesc *>(bars + 2 * NS + 2);   // [NS]
     int *sflag = reinterpret_cast<int *>(sdesc + NS);                    // [16]
     int *cum = sflag + 16;                                               // [N + 1]
     int *Ts = cum + a.N + 1;                                             // [N]
@@ -148,6 +203,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             mbar_init(smem_addr(&bars[s]), 1);
             mbar_init(smem_addr(&bars[NS + s]), C::GW);
         }
+        mbar_init(smem_addr(&bars[2 * NS]), C::NCW);  // draft block written into the ring (fused append)
         mbar_fence_init();
     }
     // rows past a short box are never written by TMA: keep them finite
@@ -217,8 +273,10 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const uint32_t empty0 = smem_addr(&bars[NS]);
     const uint32_t stage0 = smem_addr(stages);
 
+    // fused append (ripe_append_verify): does tile gt hold rows of the draft block (ring, t >= T)?
+    const bool fused = a.blk_k != nullptr;
     if (warp == C::NCW) {
-        // ================================================================ producer
+        // ================================================================ producer (one thread)
         if (lane == 0) {
             int n = seq_of(cum, N, g_begin);
             SeqGeom sg = seq_geom(Ts[n], pa);
@@ -228,7 +286,16 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             const int P0 = n * kvH + kh;
             int i = 0;
             bool ok = true;
-            for (; i < ntiles; ++i) {
+            // with a fused append, the ring tiles wait until the consumers have written the block's
+            // rows into the ring: the first ring tile of this CTA is tile sg.nd - lt (deep tiles of a
+            // head come first), so the loop below runs in two phases and stays free of that check
+            int bound = ntiles;
+            if (fused) {
+                const int first_ring = sg.nd - lt > 0 ? sg.nd - lt : 0;
+                if (first_ring < ntiles) bound = first_ring;
+            }
+            for (;;) {
+            for (; i < bound; ++i) {
                 const int s = i % NS;
                 if (i >= NS && !mbar_wait_bounded(empty0 + 8 * s, ((i / NS) - 1) & 1)) {
                     ok = false;
@@ -273,6 +340,14 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     }
                 }
             }
+            if (!ok || bound >= ntiles) break;
+            // the consumers wrote the block's rows into the ring (generic proxy) and fenced them
+            if (!mbar_wait_bounded(smem_addr(&bars[2 * NS]), 0)) {
+                ok = false;
+                break;
+            }
+            bound = ntiles;
+            }
             if (!ok) {
                 atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
                 // drain: the last issue of every stage must land before the CTA exits
@@ -282,6 +357,17 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         }
         return;  // the producer warp takes part in no consumer barrier (id 1)
     }
+
+#ifndef RIPE_NO_FUSED_APPEND
+    if (fused) {
+        // consumers, before their first tile: write the draft block's rows that this CTA's ring
+        // tiles read into the ring, fence them for the TMA (async proxy), release the producer
+        fused_block_copy<D>(a, cum, Ts, g_begin, g_end, tid, C::NCW * 32);
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&bars[2 * NS]));
+    }
+#endif
 
     // ==================================================================== consumers
     const int tg = warp / C::GW;             // tile group: tiles i with i % TG == tg
@@ -683,6 +769,7 @@ struct Inst {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for<C>(N));
     }
     static void launch(const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
+        if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
         launch_pdl(ripe_verify_kernel<D, NQT, WR, WK, TG>, dim3(grid), dim3(C::THREADS),
                    smem_bytes_for<C>(c->N), s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
     }
@@ -737,13 +824,13 @@ static void launch_d(int qc, const ripe_cache *c, int grid, const VerifyArgs &a,
 template <class I0, class I1, class I2, class I3>
 static cudaError_t launch_raw_d(int qc, const RawVerify &rv, const VerifyArgs &a, cudaStream_t s) {
     switch (qc) {
-        case 0: return launch_pdl(ripe_verify_kernel_of<I0>(), dim3(rv.grid), dim3(I0::C::THREADS),
+        case 0: return launch_pdl(ripe_verify_kernel_of<I0>(), dim3(rv.grid < I0::C::MAX_PARTS ? rv.grid : I0::C::MAX_PARTS), dim3(I0::C::THREADS),
                                   smem_bytes_for<typename I0::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        case 1: return launch_pdl(ripe_verify_kernel_of<I1>(), dim3(rv.grid), dim3(I1::C::THREADS),
+        case 1: return launch_pdl(ripe_verify_kernel_of<I1>(), dim3(rv.grid < I1::C::MAX_PARTS ? rv.grid : I1::C::MAX_PARTS), dim3(I1::C::THREADS),
                                   smem_bytes_for<typename I1::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        case 2: return launch_pdl(ripe_verify_kernel_of<I2>(), dim3(rv.grid), dim3(I2::C::THREADS),
+        case 2: return launch_pdl(ripe_verify_kernel_of<I2>(), dim3(rv.grid < I2::C::MAX_PARTS ? rv.grid : I2::C::MAX_PARTS), dim3(I2::C::THREADS),
                                   smem_bytes_for<typename I2::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        default: return launch_pdl(ripe_verify_kernel_of<I3>(), dim3(rv.grid), dim3(I3::C::THREADS),
+        default: return launch_pdl(ripe_verify_kernel_of<I3>(), dim3(rv.grid < I3::C::MAX_PARTS ? rv.grid : I3::C::MAX_PARTS), dim3(I3::C::THREADS),
                                    smem_bytes_for<typename I3::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
     }
 }
@@ -765,6 +852,9 @@ int verify_rows_for(int Mq) { return 8 << qcfg_of(Mq); }
 
 int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     VerifyArgs a;
+    a.blk_k = a.blk_v = nullptr;
+    a.ring_k = a.ring_v = nullptr;
+    a.max_T = 0;
     a.q = static_cast<const __nv_bfloat16 *>(rv.q);
     a.out = static_cast<__nv_bfloat16 *>(rv.out);
     a.lse = rv.lse;
@@ -799,8 +889,10 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
 static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s);
 
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,
-                  cudaStream_t s) {
+                  cudaStream_t s, const void *blk_k, const void *blk_v) {
     VerifyArgs a;
+    a.blk_k = static_cast<const uint4 *>(blk_k);
+    a.blk_v = static_cast<const uint4 *>(blk_v);
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
@@ -827,6 +919,7 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                        float *lse, float scale, cudaStream_t s) {
     VerifyArgs a;
+    a.blk_k = a.blk_v = nullptr;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
@@ -848,6 +941,9 @@ int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position
 }
 
 static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s) {
+    a.ring_k = reinterpret_cast<uint4 *>(c->Kw);
+    a.ring_v = reinterpret_cast<uint4 *>(c->Vw);
+    a.max_T = c->max_T;
     a.T = c->T_dev;
     a.part_o = c->part_o;
     a.part_ml = c->part_ml;

@@ -22,7 +22,7 @@ EXPORTS = (
     "ripe_cache_alloc", "ripe_cache_free", "ripe_load_prefix", "ripe_append_block",
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
-    "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave",
+    "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave", "ripe_append_verify",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "ripe_strerror": ([i], ctypes.c_char_p),
             "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
             "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
+            "ripe_append_verify": ([vp, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -152,6 +153,12 @@ def ripe_verify_attn(h, layer, r, q, out, lse=None, scale=1.0, stream=None):
     _check(lib().ripe_verify_attn(h, layer, r, ctypes.c_void_p(q), ctypes.c_void_p(out),
                                   ctypes.c_void_p(lse or 0), float(scale), _stream(stream)),
            "ripe_verify_attn")
+
+
+def ripe_append_verify(h, layer, r, B, k, v, q, out, lse=None, scale=1.0, stream=None):
+    _check(lib().ripe_append_verify(h, layer, r, B, ctypes.c_void_p(k), ctypes.c_void_p(v), ctypes.c_void_p(q),
+                                    ctypes.c_void_p(out), ctypes.c_void_p(lse or 0), float(scale),
+                                    _stream(stream)), "ripe_append_verify")
 
 
 def ripe_verify_attn_wave(h, layer, loop_of_position, q, out, lse=None, scale=1.0, stream=None):
@@ -258,6 +265,22 @@ class RipeCache:
         op = _dev(out, torch.bfloat16, shape, "out").value
         lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
         ripe_verify_attn(self.handle, layer, r, qp, op, lp, scale, stream)
+        return out
+
+    def append_verify(self, layer, r, k, v, q, out=None, lse=None, scale=1.0, stream=None):
+        """append_block(layer, r, k, v) + verify_attn(layer, r, q) in one launch."""
+        import torch
+        B = q.shape[1]
+        kshape = (self.N, B, self.kvH, self.d)
+        shape = (self.N, B, self.Hq, self.d)
+        kp = _dev(k, torch.bfloat16, kshape, "k").value
+        vp = _dev(v, torch.bfloat16, kshape, "v").value
+        qp = _dev(q, torch.bfloat16, shape, "q").value
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+        op = _dev(out, torch.bfloat16, shape, "out").value
+        lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
+        ripe_append_verify(self.handle, layer, r, B, kp, vp, qp, op, lp, scale, stream)
         return out
 
     def verify_attn_wave(self, layer, loop_of_position, q, out=None, lse=None, scale=1.0, stream=None):

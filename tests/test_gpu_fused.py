@@ -1,0 +1,50 @@
+"""ripe_append_verify == ripe_append_block + ripe_verify_attn, bit for bit: the outputs of every
+call and the cache state after each commit, over several decode steps with ragged accepted
+lengths (ring wrap-around, eviction, all three layouts)."""
+import numpy as np
+import pytest
+import torch
+
+from harness import dev_to_bits
+from self_speculative_decode_b200.ripe import RipeCache
+from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("W,B,g,d", [(16, 8, 1, 96), (5, 6, 2, 64), (0, 4, 4, 128), (10 ** 6, 8, 1, 96),
+                                     (64, 8, 4, 128)])
+def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, cuda_device):
+    N, L, kvH, R, T0, steps = 3, 2, 3, 4, 90, 6
+    max_T = T0 + B * (steps + 1)
+    src = PlaneSource(N, kvH, d, R, T0, 0.88, 31, backend="torch", device=cuda_device)
+    caches = [RipeCache(N, L, kvH * g, kvH, d, R, W, max_T, B) for _ in range(2)]
+    T = [T0, 7, 45]
+    for layer in range(L):
+        s = PlaneSource(N, kvH, d, R, T0, 0.88, 31, layer=layer, backend="torch", device=cuda_device)
+        for pl in range(R):
+            k, v = s.plane(pl, "K"), s.plane(pl, "V")
+            for c in caches:
+                c.load_prefix(layer, pl, T, k, v)
+    acc = acceptance_draws(5, steps, N, B)
+    for step in range(steps):
+        for r in range(R):
+            for layer in range(L):
+                kb, vb = src.block(step * L + layer, r, B, "K"), src.block(step * L + layer, r, B, "V")
+                q = src.queries(r, B, kvH * g, step * L + layer)
+                caches[0].append_block(layer, r, kb, vb)
+                a = caches[0].verify_attn(layer, r, q)
+                b = caches[1].append_verify(layer, r, kb, vb, q)
+                assert torch.equal(a, b), (step, r, layer)
+        for c in caches:
+            c.commit(acc[step])
+        for n in range(N):
+            for layer in range(L):
+                ka, va, pa = caches[0].export(n, layer)
+                kb_, vb_, pb = caches[1].export(n, layer)
+                assert torch.equal(pa, pb)
+                assert np.array_equal(dev_to_bits(ka), dev_to_bits(kb_))
+                assert np.array_equal(dev_to_bits(va), dev_to_bits(vb_))
+    for c in caches:
+        assert c.device_error() == 0
+        c.close()
