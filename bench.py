@@ -67,6 +67,18 @@ def verify_bytes(cfg, T_list, r):
     return keys * row + qo
 
 
+DRAFT_LOOPS = 4  # draft depth of the timed draft phase: loops 0..3 of 32
+
+
+def draft_bytes(cfg, T_list, r, j, W):
+    """Algorithmic bytes of one draft step (block position j at loop r): one plane per key
+    t <= T + j, the deepest-plane reads of window keys older than W for that query, the
+    query and the output."""
+    row = 4 * cfg["kvH"] * cfg["d"]
+    keys = sum(T + j + 1 + dual_keys(T, W, j + 1, cfg["R"], r) for T in T_list)
+    return keys * row + 2 * cfg["N"] * cfg["Hq"] * cfg["d"] * 2
+
+
 def sources_digest():
     """sha256 over the library's CUDA sources and C header (ties an ncu capture to a kernel version)."""
     import glob
@@ -195,12 +207,13 @@ def gpu_id(index):
 class Workload:
     """One cache with a loaded prefix, the step's inputs in HBM, and its CUDA graphs."""
 
-    def __init__(self, cfg, layout, total_steps, seed, device):
+    def __init__(self, cfg, layout, total_steps, seed, device, fused=False):
         import torch
         from self_speculative_decode_b200.ripe import RipeCache
         from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
 
         self.cfg, self.layout, self.device = cfg, layout, device
+        self.fused = fused
         N, L, Hq, kvH, d, R, T, B = (cfg[k] for k in ("N", "L", "Hq", "kvH", "d", "R", "T", "B"))
         self.max_T = T + B * (total_steps + 4)
         W = {"ripe": cfg["W"], "full": self.max_T, "deepest": 0}[layout]
@@ -235,9 +248,12 @@ class Workload:
             for layer in range(cfg["L"]):
                 if verify_only:
                     c.verify_attn(layer, r, self.q[layer, r], out=self.out[layer, r])
-                else:  # append plane r of the block and verify at loop r: one launch
+                elif self.fused:  # append plane r of the block and verify at loop r: one launch
                     c.append_verify(layer, r, self.k[layer, r], self.v[layer, r], self.q[layer, r],
                                     out=self.out[layer, r])
+                else:
+                    c.append_block(layer, r, self.k[layer, r], self.v[layer, r])
+                    c.verify_attn(layer, r, self.q[layer, r], out=self.out[layer, r])
 
     def capture(self):
         import torch
@@ -316,7 +332,7 @@ def step_bytes(cfg, T_start, acc_rows):
 
 def bench_layout(cfg, layout, args, seed, device, dist_on, want_extras):
     import torch
-    wl = Workload(cfg, layout, args.warmup + 2 * args.steps + 2, seed, device)
+    wl = Workload(cfg, layout, args.warmup + 2 * args.steps + 2, seed, device, fused=args.append == "fused")
     wl.capture()
     N = cfg["N"]
     res = {}
@@ -328,6 +344,8 @@ def bench_layout(cfg, layout, args, seed, device, dist_on, want_extras):
     per_step, T_end = step_bytes(cfg, T_start, rows)
     T_check = wl.cache.sync_lengths()
     assert T_check == T_end, (T_check, T_end)
+    if want_extras:
+        res["draft"] = draft_timing(wl, args, dist_on)
     nbytes = sum(per_step)
     res.update(ms_per_step=ms / args.steps, bytes_per_step=nbytes / args.steps,
                gbs=nbytes / (ms * 1e-3) / 1e9,
@@ -392,6 +410,36 @@ def wave_timing(wl, args, dist_on):
     us = ms * 1e3 / (reps * cfg["L"])
     nbytes = wave_bytes(cfg, T_now, wl.W)
     return dict(us_per_call=us, bytes_per_call=nbytes, gbs=nbytes / (us * 1e-6) / 1e9, loops=loops)
+
+
+def draft_timing(wl, args, dist_on):
+    """The draft phase of one block as a CUDA graph: for each block position j, every layer at
+    loops 0 .. DRAFT_LOOPS-1 writes plane r of position j and attends its query (B = 1)."""
+    import torch
+    cfg, c = wl.cfg, wl.cache
+    L, B, rd = cfg["L"], cfg["B"], min(DRAFT_LOOPS, cfg["R"])
+    dk = [[[wl.k[layer, r][:, j:j + 1].contiguous() for j in range(B)] for r in range(rd)] for layer in range(L)]
+    dv = [[[wl.v[layer, r][:, j:j + 1].contiguous() for j in range(B)] for r in range(rd)] for layer in range(L)]
+    dq = [[[wl.q[layer, r][:, j:j + 1].contiguous() for j in range(B)] for r in range(rd)] for layer in range(L)]
+    dout = torch.empty_like(dq[0][0][0])
+    n0 = c.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for j in range(B):
+            for layer in range(L):
+                for r in range(rd):
+                    c.draft_attn(layer, r, j, dk[layer][r][j], dv[layer][r][j], dq[layer][r][j], out=dout)
+    launches = c.launch_count() - n0
+    reps = max(3, args.steps)
+    g.replay()
+    ms = max_over_ranks(time_region(lambda: [g.replay() for _ in range(reps)], dist_on), dist_on)
+    T_now = c.sync_lengths()
+    nbytes = sum(draft_bytes(cfg, T_now, r, j, wl.W) for j in range(B) for r in range(rd)) * L
+    phase_ms = ms / reps
+    return dict(loops=rd, calls_per_block=launches, ms_per_block=phase_ms,
+                us_per_call=phase_ms * 1e3 / launches, bytes_per_call=nbytes / launches,
+                gbs=nbytes / (phase_ms * 1e-3) / 1e9,
+                drafted_tokens_per_s=cfg["N"] * B / (phase_ms * 1e-3))
 
 
 def e2e_steps(wl, args, dist_on):
@@ -516,6 +564,8 @@ def main():
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many verify calls of layer 0 (for ncu captures) and exit")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--append", default="separate", choices=["separate", "fused"],
+                    help="block append as its own launch before each verify, or inside it (ripe_append_verify)")
     ap.add_argument("--seed", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -570,7 +620,9 @@ def main():
         "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg["workload"], "layout": main_l,
-                   "step": "R*L x fused (append plane r + verify at loop r) + commit/evict, CUDA graph",
+                   "step": ("R*L x (append plane r + verify at loop r" +
+                            (", one launch" if args.append == "fused" else ", two launches") +
+                            ") + commit/evict, CUDA graph"),
                    "T_range": m["T_range"], "l2": "inputs larger than L2 (every step reads the whole cache)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": 100.0 * m["gbs"] / peak,
@@ -598,6 +650,13 @@ def main():
             "ripe_gbs": wr["gbs"], "full_gbs": wf["gbs"],
             "note": "one call per layer verifies every block position at its own loop; the deepest "
                     "region is read once for all loops, the window once per loop"}
+    if "draft" in m:
+        d = m["draft"]
+        line["draft_phase"] = dict(d, pct_of_hbm_peak=100.0 * d["gbs"] / peak,
+                                   cycle_ms=d["ms_per_block"] + m["ms_per_step"],
+                                   note=f"draft-then-verify: B positions drafted one at a time at loops "
+                                        f"0..{d['loops'] - 1} of every layer (ripe_draft_attn, B=1 decode "
+                                        f"shape), then the step verifies the block at all R loops")
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         gbs, calls, sec, threads = oracle_sample(cfg, args.cpu_seconds)
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",

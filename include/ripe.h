@@ -159,6 +159,27 @@ int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, 
                        const void *q, void *out, float *lse, float scale, void *stream);
 
 /*
+ * One step of the draft phase: block position j at loop r, written and attended in one launch.
+ * Draft-then-verify builds the draft block one position at a time at a shallow depth, then
+ * checks the whole block at full depth (RIPE abstract, first sentence; WaveFront write-up,
+ * section on drafting and checking in one pass).  Plane r of position T_n + j is written to
+ * ring slot (T_n + j) mod S from k, v; then the query of that position attends over keys
+ * t <= T_n + j with the plane rule of ripe_verify_attn for query p = T_n + j: the draft
+ * positions 0 .. j at plane r, the window at plane r, older keys at the deepest plane.
+ * The result equals row j of ripe_verify_attn over a block whose plane r holds the same rows.
+ *   j        0 .. max_B - 1; positions 0 .. j-1 of plane r must have been drafted since the
+ *            last commit (else RIPE_ESTATE); redrafting j makes later drafted positions stale
+ *   k, v     device bf16 [batch][1][kv_heads][d], plane r of position j
+ *   q, out   device bf16 [batch][1][q_heads][d];  lse  device fp32 [batch][1][q_heads] or NULL
+ * Requires no verification block in flight (the first ripe_append_block of the block ends the
+ * draft phase; RIPE_ESTATE) and T_n + j + 1 <= max_T (RIPE_ECAPACITY).  ripe_commit (or
+ * ripe_commit_device) ends the draft phase of the block; ripe_load_prefix is refused while a
+ * draft is in flight.
+ */
+int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, const void *v,
+                    const void *q, void *out, float *lse, float scale, void *stream);
+
+/*
  * Verification attention with a loop per block position: block position j is evaluated
  * exactly as ripe_verify_attn(.., loop_of_position[j], ..) would evaluate it.  This is the
  * shape of a wavefront schedule, where one batched pass of the looped block holds positions

@@ -22,6 +22,10 @@ Contents
   * ``verify_wave``    a loop per block position: each position evaluated as the
                        single-loop verification at its own loop (definition by
                        composition).
+  * ``OracleCache.draft``  one draft-phase step: plane r of block position j stored,
+                       then the query of that position attends with the verification
+                       rule for p = T + j (draft-then-verify builds the block one
+                       position at a time at a shallow loop).
 Every function here is pinned by ``tests/test_oracle_*.py``; none is "parity
 unpinned".
 """
@@ -167,6 +171,7 @@ class OracleCache:
         self.T = np.zeros(N, dtype=np.int64)
         self.B = 0
         self.appended = np.zeros((L, R), dtype=bool)
+        self.drafted = np.zeros((L, R), dtype=np.int64)   # draft positions stored per plane
         self.present = np.zeros((L, R, N, max_T), dtype=bool)
         self._K = {}
         self._V = {}
@@ -191,7 +196,7 @@ class OracleCache:
     def load_prefix(self, layer, plane, T, k, v):
         """Store what RIPE keeps of one plane of a prefix: k, v bits [N][kvH][>=T][d]."""
         T = np.asarray(T, dtype=np.int64)
-        if self.B:
+        if self.B or self.drafted.any():
             raise RuntimeError("load_prefix with a draft block in flight")
         if self._prefix_set and not np.array_equal(T, self.T):
             raise ValueError("prefix lengths differ between calls")
@@ -233,9 +238,10 @@ class OracleCache:
             raise RuntimeError("commit before every plane of the block was appended")
         if np.any(a < 0) or np.any(a > self.B):
             raise ValueError("accepted length out of range")
+        span = max(self.B, int(self.drafted.max()))   # drafts past the block are discarded too
         for n in range(self.N):
             t0 = int(self.T[n])
-            rej = slice(t0 + int(a[n]), t0 + self.B)
+            rej = slice(t0 + int(a[n]), t0 + span)
             self.present[:, :, n, rej] = False
             for store in (self._K, self._V):
                 for arr in store.values():
@@ -248,6 +254,44 @@ class OracleCache:
                     arr[n, :, old] = 0
         self.B = 0
         self.appended[:] = False
+        self.drafted[:] = 0
+
+    # -- draft phase --------------------------------------------------------------
+    def draft(self, layer, r, j, k, v, q_bits, g, scale=1.0):
+        """Draft step at loop r for block position j of every sequence.
+
+        Stores plane r of position T_n + j (k, v bits [N][1][kvH][d]); positions after j of
+        that plane become stale.  Then the query q_bits [N][1][Hq][d] of position p = T_n + j
+        attends over keys t <= p: the definition of ``verify`` with a block of j + 1
+        positions, row j (the drafts 0 .. j at plane r, the window from p, older keys at the
+        deepest plane).  Returns (out [N][1][Hq][d], lse [N][1][Hq]) in fp64.
+        """
+        if self.B:
+            raise RuntimeError("draft step with a verification block in flight")
+        if j < 0 or j > self.drafted[layer, r]:
+            raise RuntimeError("draft positions of a plane are written in order")
+        if np.any(self.T + j + 1 > self.max_T):
+            raise ValueError("capacity")
+        keep = self._keeps(r)
+        for n in range(self.N):
+            t = int(self.T[n]) + j
+            stale = slice(t + 1, int(self.T[n]) + int(self.drafted[layer, r]))
+            self.present[layer, r, n, stale] = False
+            if keep:
+                for store, x in ((self._K, k), (self._V, v)):
+                    arr = self._arr(store, layer, r)
+                    arr[n, :, t] = x[n, 0]
+                    arr[n, :, stale] = 0
+            self.present[layer, r, n, t] = True
+        self.drafted[layer, r] = j + 1
+        if not (keep and self._keeps(self.R - 1)):
+            raise RuntimeError("a draft step needs the values of planes r and R-1")
+        Kr, Vr, Kl, Vl, _ = self.verify_inputs(layer, r)
+        qb = bf16_to_f64(q_bits)
+        qfull = np.zeros((self.N, j + 1) + qb.shape[2:])
+        qfull[:, j] = qb[:, 0]
+        out, lse = verify(self.T, j + 1, r, self.R, self.W, g, Kr, Vr, Kl, Vl, qfull, scale, self.mode)
+        return out[:, j:j + 1], lse[:, j:j + 1]
 
     # -- queries ----------------------------------------------------------------
     def stored_position_planes(self, layer, n):

@@ -81,6 +81,12 @@ struct DeviceGuard {
     }
 };
 
+bool any_drafted(const ripe_cache *c) {
+    for (size_t i = 0; i < c->drafted.size(); ++i)
+        if (c->drafted[i]) return true;
+    return false;
+}
+
 bool all_appended(const ripe_cache *c) {
     for (size_t i = 0; i < c->appended.size(); ++i)
         if (!c->appended[i]) return false;
@@ -128,6 +134,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     c->T.assign(batch, 0);
     c->B_cur = 0;
     c->appended.assign(static_cast<size_t>(layers) * loops, 0);
+    c->drafted.assign(static_cast<size_t>(layers) * loops, 0);
     c->prefix_set = false;
     c->synced = true;
     c->kv_bytes = c->scratch_bytes = 0;
@@ -189,7 +196,7 @@ int ripe_cache_free(ripe_cache_t *c) {
 int ripe_load_prefix(ripe_cache_t *c, int layer, int plane, const int32_t *T, const void *k, const void *v,
                      int64_t ld_t, void *stream) {
     if (!c || !T || !k || !v || layer < 0 || layer >= c->L || plane < 0 || plane >= c->R) return RIPE_EINVAL;
-    if (c->B_cur != 0 || !c->synced) return RIPE_ESTATE;
+    if (c->B_cur != 0 || !c->synced || any_drafted(c)) return RIPE_ESTATE;
     int Tmax = 0;
     for (int n = 0; n < c->N; ++n) {
         if (T[n] < 0) return RIPE_EINVAL;
@@ -256,6 +263,24 @@ int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, 
     return RIPE_OK;
 }
 
+int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, const void *v, const void *q,
+                    void *out, float *lse, float scale, void *stream) {
+    if (!c || !k || !v || !q || !out || layer < 0 || layer >= c->L || r < 0 || r >= c->R || j < 0 ||
+        j >= c->max_B)
+        return RIPE_EINVAL;
+    const size_t idx = static_cast<size_t>(layer) * c->R + r;
+    if (c->B_cur != 0 || j > c->drafted[idx]) return RIPE_ESTATE;
+    for (int n = 0; n < c->N; ++n)
+        if (c->T[n] + j + 1 > c->max_T) return RIPE_ECAPACITY;
+    DeviceGuard g(c->device);
+    if (!g.ok) return RIPE_ECUDA;
+    const int st = launch_draft(c, layer, r, j, k, v, q, out, lse, scale, static_cast<cudaStream_t>(stream));
+    if (st != RIPE_OK) return st;
+    c->drafted[idx] = j + 1;  // a later position of this plane is stale once j is redrafted
+    c->prefix_set = true;
+    return RIPE_OK;
+}
+
 int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                           float *lse, float scale, void *stream) {
     if (!c || !loop_of_position || !q || !out || layer < 0 || layer >= c->L) return RIPE_EINVAL;
@@ -282,6 +307,7 @@ int ripe_commit(ripe_cache_t *c, const int32_t *accepted_len, void *stream) {
     for (int n = 0; n < c->N; ++n) c->T[n] += accepted_len[n];
     c->B_cur = 0;
     std::fill(c->appended.begin(), c->appended.end(), 0);
+    std::fill(c->drafted.begin(), c->drafted.end(), 0);
     return RIPE_OK;
 }
 
@@ -296,6 +322,7 @@ int ripe_commit_device(ripe_cache_t *c, const int32_t *accepted_len, void *strea
     c->synced = false;
     c->B_cur = 0;
     std::fill(c->appended.begin(), c->appended.end(), 0);
+    std::fill(c->drafted.begin(), c->drafted.end(), 0);
     return RIPE_OK;
 }
 

@@ -52,6 +52,7 @@ struct ripe_cache {
     std::vector<int32_t> T;   // committed lengths (an upper bound when !synced)
     int B_cur;                // block in flight (0 = none)
     std::vector<uint8_t> appended;  // [L][R] planes of the block appended
+    std::vector<int> drafted;       // [L][R] draft positions written at each plane (before the block)
     bool prefix_set, synced;
     int64_t kv_bytes, scratch_bytes;
     int64_t launches;
@@ -285,6 +286,8 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 // ---------------------------------------------------------------- launchers (defined per .cu)
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
                   float scale, cudaStream_t s, const void *blk_k = nullptr, const void *blk_v = nullptr);
+int launch_draft(ripe_cache *c, int layer, int r, int j, const void *k, const void *v, const void *q, void *out,
+                 float *lse, float scale, cudaStream_t s);
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q,
                        void *out, float *lse, float scale, cudaStream_t s);
 int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const void *v,

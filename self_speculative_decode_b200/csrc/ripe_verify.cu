@@ -45,6 +45,9 @@ struct VerifyArgs {
     uint32_t *err;
     PlanArgs plan;
     int N, kvH, g, Hq, B, R, layer, Mq, min_chunk;
+    // queries: block positions j0 .. j0 + qB - 1 (q, out, lse and the fused block hold qB rows
+    // per sequence); a verification has j0 = 0, qB = B, a draft step j0 = its position, qB = 1
+    int j0, qB;
     int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
     float scale_log2;
     // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
@@ -123,9 +126,15 @@ __device__ __forceinline__ int pair_of(const int *cum, int N, int kvH, int gt) {
     return n * kvH + (gt - cum[n]) / tot;
 }
 
-// Fused append: the rows of the draft block (positions >= T) inside this CTA's ring tiles are
-// copied from the caller's block K/V [N][B][kvH][d] into ring plane r.  No other tile of the
-// launch reads those slots.  Kept out of line: it runs once per CTA, away from the tile loop.
+// Ring tile (index within the pair's list) holding position pos of the single-loop ring [D, T + B).
+__device__ __forceinline__ int ring_tile_of(const SeqGeom &sg, const PlanArgs &pa, int pos) {
+    const int o = pos - sg.D;
+    return sg.nd + (o < sg.ring_first ? o / pa.ring_box : sg.nr1 + (o - sg.ring_first) / pa.ring_box);
+}
+
+// Fused append: the rows of the draft block (positions >= T + j0) inside this CTA's ring tiles
+// are copied from the caller's block K/V [N][qB][kvH][d] into ring plane r.  No other tile of
+// the launch reads those slots.  Kept out of line: it runs once per CTA, away from the tile loop.
 template <int D>
 __device__ __noinline__ void fused_block_copy(const VerifyArgs &a, const int *cum, const int *Ts, int g_begin,
                                               int g_end, int tid, int nthreads) {
@@ -141,17 +150,18 @@ __device__ __noinline__ void fused_block_copy(const VerifyArgs &a, const int *cu
             continue;
         }
         const int start = cum[n] + kh * sg.total;
-        for (int lt = sg.nd; lt < sg.nd + sg.nr; ++lt) {
+        const int first = sg.T + a.j0;  // first position written by this call
+        const int lt_hi = ring_tile_of(sg, pa, sg.T + a.B - 1);
+        for (int lt = ring_tile_of(sg, pa, first); lt <= lt_hi; ++lt) {
             const int gt = start + lt;
             if (gt < g_begin || gt >= g_end) continue;
             const Tile t = tile_at(sg, lt, pa);
-            if (t.t0 + t.cnt <= sg.T) continue;
-            const int r0 = t.t0 > sg.T ? t.t0 : sg.T;
+            const int r0 = t.t0 > first ? t.t0 : first;
             const int rows = t.t0 + t.cnt - r0;
             for (int e = tid; e < rows * d8; e += nthreads) {
                 const int row = e / d8, c8 = e - (e / d8) * d8;
                 const int tpos = r0 + row;
-                const size_t src = ((static_cast<size_t>(n) * a.B + (tpos - sg.T)) * kvH + kh) * d8 + c8;
+                const size_t src = ((static_cast<size_t>(n) * a.qB + (tpos - first)) * kvH + kh) * d8 + c8;
                 const size_t dst = ((((static_cast<size_t>(a.layer) * N + n) * a.R + t.plane) * kvH + kh) *
                                         pa.ring_slots + (t.y + (tpos - t.t0))) * d8 + c8;
                 a.ring_k[dst] = a.blk_k[src];
@@ -161,11 +171,36 @@ __device__ __noinline__ void fused_block_copy(const VerifyArgs &a, const int *cu
     }
 }
 
-template <int D, int NQT, int WR, int WK, int TG>
-__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS, 1)
+// Fused append: index (within the chunk) of the first tile holding a row the launch writes
+// (positions T + j0 .. T + B - 1 of a pair), or ntiles if the chunk has none.  The chunk
+// starts at tile lt of pair (n, kh) with geometry sg.
+__device__ __noinline__ int first_written_tile(SeqGeom sg, int lt, int n, int kh, int ntiles, const int *Ts,
+                                               const VerifyArgs &a) {
+    const PlanArgs &pa = a.plan;
+    int i = 0;
+    while (i < ntiles) {
+        const int lo = ring_tile_of(sg, pa, sg.T + a.j0), hi = ring_tile_of(sg, pa, sg.T + a.B - 1);
+        if (lt <= hi) {
+            const int at = i + (lo > lt ? lo - lt : 0);
+            return at < ntiles ? at : ntiles;
+        }
+        i += sg.total - lt;
+        lt = 0;
+        if (++kh == a.kvH) {
+            kh = 0;
+            if (++n >= a.N) break;
+            sg = seq_geom(Ts[n], pa);
+        }
+    }
+    return ntiles;
+}
+
+// FUSED adds one warp after the producer that writes the draft block's rows into the ring.
+template <int D, int NQT, int WR, int WK, int TG, bool FUSED>
+__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS + (FUSED ? 32 : 0), 1)
 ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_constant__ CUtensorMap tmVd,
                    const __grid_constant__ CUtensorMap tmKw, const __grid_constant__ CUtensorMap tmVw,
-                   const VerifyArgs a) {
+                   const __grid_constant__ VerifyArgs a) {
     using C = VCfg<D, NQT, WR, WK, TG>;
     constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
@@ -203,7 +238,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             mbar_init(smem_addr(&bars[s]), 1);
             mbar_init(smem_addr(&bars[NS + s]), C::GW);
         }
-        mbar_init(smem_addr(&bars[2 * NS]), C::NCW);  // draft block written into the ring (fused append)
+        if (FUSED) mbar_init(smem_addr(&bars[2 * NS]), 1);  // draft block written into the ring
         mbar_fence_init();
     }
     // rows past a short box are never written by TMA: keep them finite
@@ -248,24 +283,43 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         if (lane == 0) {
             int ch = cdiv(total, static_cast<int>(gridDim.x));
             if (ch < a.min_chunk) ch = a.min_chunk;
+            int pieces = 0;
             if (same) {
                 // cut at (sequence, kv head) boundaries when that costs at most kSwitchTiles
                 // tiles per CTA: a CTA then never switches to another head mid-stream
                 if (ch < tot0) {
-                    const int ca = cdiv(tot0, tot0 / ch);
-                    if (ca <= ch + kSwitchTiles) ch = ca;
+                    // several CTAs per head: `pieces` equal pieces of each head, CTA c taking
+                    // piece c % pieces of head c / pieces
+                    int P = static_cast<int>(gridDim.x) / (N * kvH);
+                    if (P > tot0 / a.min_chunk) P = tot0 / a.min_chunk;
+                    if (P >= 1) {
+                        const int ca = cdiv(tot0, P);
+                        if (ca <= ch + kSwitchTiles) {
+                            ch = ca;
+                            pieces = P;
+                        }
+                    }
                 } else {
                     const int ca = cdiv(ch, tot0) * tot0;
                     if (ca <= ch + kSwitchTiles) ch = ca;
                 }
             }
             sflag[6] = ch;
+            sflag[7] = pieces;
         }
     }
     __syncthreads();
     const int chunk = sflag[6];
-    const int g_begin = blockIdx.x * chunk;
-    const int g_end = min(total, g_begin + chunk);
+    const int pieces = sflag[7];  // 0: contiguous chunks of the whole tile list
+    int g_begin, g_end;
+    if (pieces) {
+        const int tot0 = cum[1] / kvH, h = blockIdx.x / pieces;
+        g_begin = h * tot0 + (blockIdx.x - h * pieces) * chunk;
+        g_end = min(min(g_begin + chunk, (h + 1) * tot0), total);
+    } else {
+        g_begin = blockIdx.x * chunk;
+        g_end = min(total, g_begin + chunk);
+    }
     if (g_begin >= g_end) return;
     const int ntiles = g_end - g_begin;
 
@@ -273,8 +327,20 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const uint32_t empty0 = smem_addr(&bars[NS]);
     const uint32_t stage0 = smem_addr(stages);
 
-    // fused append (ripe_append_verify): does tile gt hold rows of the draft block (ring, t >= T)?
-    const bool fused = a.blk_k != nullptr;
+    // FUSED (ripe_append_verify): the consumers first write the draft block into the ring; a
+    // separate instantiation so that plain verification carries none of that code
+    constexpr bool fused = FUSED;
+    if constexpr (fused) {
+        if (warp == C::NCW + 1) {
+            // the copy warp: write the draft block's rows that this CTA's tiles read into the
+            // ring, fence them for the TMA (async proxy), release the producer
+            fused_block_copy<D>(a, cum, Ts, g_begin, g_end, lane, 32);
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&bars[2 * NS]));
+            return;
+        }
+    }
     if (warp == C::NCW) {
         // ================================================================ producer (one thread)
         if (lane == 0) {
@@ -286,14 +352,11 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             const int P0 = n * kvH + kh;
             int i = 0;
             bool ok = true;
-            // with a fused append, the ring tiles wait until the consumers have written the block's
-            // rows into the ring: the first ring tile of this CTA is tile sg.nd - lt (deep tiles of a
-            // head come first), so the loop below runs in two phases and stays free of that check
+            // with a fused append, the tiles holding the rows this launch writes wait until the
+            // consumers have written them: the loop below runs in two phases, up to the first such
+            // tile of the chunk and from it, and stays free of a per-tile check
             int bound = ntiles;
-            if (fused) {
-                const int first_ring = sg.nd - lt > 0 ? sg.nd - lt : 0;
-                if (first_ring < ntiles) bound = first_ring;
-            }
+            if (fused) bound = first_written_tile(sg, lt, n, kh, ntiles, Ts, a);
             for (;;) {
             for (; i < bound; ++i) {
                 const int s = i % NS;
@@ -331,9 +394,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     const int p_last = pair_of(cum, N, kvH, g_end - 1);
                     for (int p = P0 + 1; p <= p_last; ++p) {
                         const int pn = p / kvH, pk = p - pn * kvH;
-                        for (int j = 0; j < a.B; ++j) {
+                        for (int j = 0; j < a.qB; ++j) {
                             const char *row = reinterpret_cast<const char *>(
-                                a.q + ((static_cast<size_t>(pn) * a.B + j) * a.Hq + pk * a.g) * D);
+                                a.q + ((static_cast<size_t>(pn) * a.qB + j) * a.Hq + pk * a.g) * D);
                             for (int off = 0; off < a.g * D * 2; off += 128)
                                 asm volatile("prefetch.global.L2 [%0];" ::"l"(row + off));
                         }
@@ -358,16 +421,6 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         return;  // the producer warp takes part in no consumer barrier (id 1)
     }
 
-#ifndef RIPE_NO_FUSED_APPEND
-    if (fused) {
-        // consumers, before their first tile: write the draft block's rows that this CTA's ring
-        // tiles read into the ring, fence them for the TMA (async proxy), release the producer
-        fused_block_copy<D>(a, cum, Ts, g_begin, g_end, tid, C::NCW * 32);
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&bars[2 * NS]));
-    }
-#endif
 
     // ==================================================================== consumers
     const int tg = warp / C::GW;             // tile group: tiles i with i % TG == tg
@@ -385,7 +438,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         for (int e = 0; e < 2; ++e) {
             const int i = C::NQ * rg + 8 * nq + 2 * c4 + e;
             qvalid[nq][e] = i < a.Mq;
-            jq[nq][e] = qvalid[nq][e] ? i / a.g : a.B - 1;
+            jq[nq][e] = qvalid[nq][e] ? a.j0 + i / a.g : a.B - 1;
             lq[nq][e] = qvalid[nq][e] ? pa.jloop[jq[nq][e]] : -1;
         }
     // ldmatrix lane geometry (64-byte swizzle: 16-byte chunk ^= (row >> 1) & 3)
@@ -426,7 +479,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             if (i < a.Mq) {
                 const int j = i / a.g, hg = i - j * a.g;
                 qp = reinterpret_cast<const uint32_t *>(
-                    a.q + ((static_cast<size_t>(n) * a.B + j) * a.Hq + kh * a.g + hg) * D);
+                    a.q + ((static_cast<size_t>(n) * a.qB + j) * a.Hq + kh * a.g + hg) * D);
             }
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
@@ -434,6 +487,19 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 qb[ks][nq][1] = qp ? __ldg(qp + 8 * ks + 4 + c4) : 0u;
             }
         }
+    };
+
+    // the CTAs holding tiles of pair p: c_first .. c_first + nparts - 1 (returns nparts)
+    auto parts_of = [&](int p, int &c_first) -> int {
+        const int n = p / kvH, kh = p - (p / kvH) * kvH;
+        const int tot_n = (cum[n + 1] - cum[n]) / kvH;
+        if (pieces) {
+            c_first = p * pieces;
+            return cdiv(tot_n, chunk);
+        }
+        const int start = cum[n] + kh * tot_n;
+        c_first = start / chunk;
+        return (start + tot_n - 1) / chunk - c_first + 1;
     };
 
     // ---------------------------------------------------------------- finalize one pair
@@ -479,10 +545,8 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         }
         named_bar_sync(1, nct);
         const bool abort_now = *reinterpret_cast<volatile int *>(&sflag[1]) != 0;
-        const int tot_n = (cum[n + 1] - cum[n]) / kvH;
-        const int start = cum[n] + kh * tot_n;
-        const int c_first = start / chunk, c_last = (start + tot_n - 1) / chunk;
-        const int nparts = c_last - c_first + 1;
+        int c_first;
+        const int nparts = parts_of(p, c_first);
         const bool sole = nparts == 1;
         // per query row: the maximum over the warps that saw it, their weights and the sum
         for (int i = tid; i < C::ROWS; i += nct) {
@@ -522,7 +586,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 }
             if (sole) {
                 const int j = i / a.g, h = kh * a.g + (i - j * a.g);
-                const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
+                const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
                 a.out[orow * D + col] = __float2bfloat16_rn(acc / fin[i * 2 + 1]);
                 if (col == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
             } else {
@@ -551,10 +615,8 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     // Runs in the CTA that arrived last, after all of its own tiles (the stage buffers are free).
     auto merge_pair = [&](int p) {
         const int n = p / kvH, kh = p - (p / kvH) * kvH;
-        const int tot_n = (cum[n + 1] - cum[n]) / kvH;
-        const int start = cum[n] + kh * tot_n;
-        const int c_first = start / chunk, c_last = (start + tot_n - 1) / chunk;
-        const int nparts = c_last - c_first + 1;
+        int c_first;
+        const int nparts = parts_of(p, c_first);
         float *pw = reinterpret_cast<float *>(stages);  // [nparts][ROWS] m, then weights
         float *pl = pw + nparts * C::ROWS;              // [nparts][ROWS] l
         float *rowML = fin;                             // [ROWS][2] final M, L
@@ -592,7 +654,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             }
             const float invL = 1.f / rowML[i * 2 + 1];
             const int j = i / a.g, h = kh * a.g + (i - j * a.g);
-            const size_t orow = (static_cast<size_t>(n) * a.B + j) * a.Hq + h;
+            const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
             __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + 4 * c4x]);
             op[0] = __floats2bfloat162_rn(acc.x * invL, acc.y * invL);
             op[1] = __floats2bfloat162_rn(acc.z * invL, acc.w * invL);
@@ -763,14 +825,19 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 template <int D, int NQT, int WR, int WK, int TG>
 struct Inst {
     using C = VCfg<D, NQT, WR, WK, TG>;
-    static constexpr auto kernel = ripe_verify_kernel<D, NQT, WR, WK, TG>;
+    static constexpr auto kernel = ripe_verify_kernel<D, NQT, WR, WK, TG, false>;
+    static constexpr auto kernel_fused = ripe_verify_kernel<D, NQT, WR, WK, TG, true>;
     static cudaError_t set_attr(int N) {
-        return cudaFuncSetAttribute(ripe_verify_kernel<D, NQT, WR, WK, TG>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes_for<C>(N));
+        const int bytes = smem_bytes_for<C>(N);
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kernel_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        return e;
     }
     static void launch(const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
         if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
-        launch_pdl(ripe_verify_kernel<D, NQT, WR, WK, TG>, dim3(grid), dim3(C::THREADS),
+        const bool fused = a.blk_k != nullptr;
+        launch_pdl(fused ? kernel_fused : kernel, dim3(grid), dim3(C::THREADS + (fused ? 32 : 0)),
                    smem_bytes_for<C>(c->N), s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
     }
 };
@@ -869,6 +936,8 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.g = rv.g;
     a.Hq = rv.Hq;
     a.B = rv.plan.B;
+    a.j0 = 0;
+    a.qB = rv.plan.B;
     a.R = rv.plan.R;
     a.layer = rv.layer;
     a.Mq = rv.plan.B * rv.g;
@@ -888,21 +957,19 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
 
 static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s);
 
-int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,
-                  cudaStream_t s, const void *blk_k, const void *blk_v) {
+// One loop r; block positions [0, B) in the tile plan, queries at positions j0 .. j0 + qB - 1.
+static int launch_single_loop(ripe_cache *c, int layer, int r, int B, int j0, int qB, const void *q, void *out,
+                              float *lse, float scale, cudaStream_t s, const void *blk_k, const void *blk_v) {
     VerifyArgs a;
     a.blk_k = static_cast<const uint4 *>(blk_k);
     a.blk_v = static_cast<const uint4 *>(blk_v);
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
-    a.T = c->T_dev;
-    a.part_o = c->part_o;
-    a.part_ml = c->part_ml;
-    a.counters = c->counters;
-    a.err = c->err_dev;
+    a.j0 = j0;
+    a.qB = qB;
     a.plan.W = c->W;
-    a.plan.B = c->B_cur;
+    a.plan.B = B;
     a.plan.R = c->R;
     a.plan.ring_slots = c->ring_slots;
     a.plan.deep_box = c->deep_box;
@@ -915,6 +982,17 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
     return launch_cache_args(c, layer, a, scale, s);
 }
 
+int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse, float scale,
+                  cudaStream_t s, const void *blk_k, const void *blk_v) {
+    return launch_single_loop(c, layer, r, c->B_cur, 0, c->B_cur, q, out, lse, scale, s, blk_k, blk_v);
+}
+
+// Draft step: position j of the block at loop r, its K/V written by the same launch.
+int launch_draft(ripe_cache *c, int layer, int r, int j, const void *k, const void *v, const void *q, void *out,
+                 float *lse, float scale, cudaStream_t s) {
+    return launch_single_loop(c, layer, r, j + 1, j, 1, q, out, lse, scale, s, k, v);
+}
+
 // Several loops in one call: block position j is verified at loop loop_of_position[j].
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                        float *lse, float scale, cudaStream_t s) {
@@ -923,6 +1001,8 @@ int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
+    a.j0 = 0;
+    a.qB = c->B_cur;
     a.plan.W = c->W;
     a.plan.B = c->B_cur;
     a.plan.R = c->R;
@@ -953,10 +1033,10 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
     a.kvH = c->kvH;
     a.g = c->g;
     a.Hq = c->Hq;
-    a.B = c->B_cur;
+    a.B = a.plan.B;
     a.R = c->R;
     a.layer = layer;
-    a.Mq = c->B_cur * c->g;
+    a.Mq = a.qB * c->g;
     a.min_chunk = RIPE_MIN_CHUNK;  // bounds the number of partials of one (sequence, kv head)
     a.has_deep = c->deep_rows > 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;

@@ -23,6 +23,7 @@ EXPORTS = (
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
     "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave", "ripe_append_verify",
+    "ripe_draft_attn",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -79,6 +80,7 @@ def lib() -> ctypes.CDLL:
             "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
             "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
             "ripe_append_verify": ([vp, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
+            "ripe_draft_attn": ([vp, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -159,6 +161,12 @@ def ripe_append_verify(h, layer, r, B, k, v, q, out, lse=None, scale=1.0, stream
     _check(lib().ripe_append_verify(h, layer, r, B, ctypes.c_void_p(k), ctypes.c_void_p(v), ctypes.c_void_p(q),
                                     ctypes.c_void_p(out), ctypes.c_void_p(lse or 0), float(scale),
                                     _stream(stream)), "ripe_append_verify")
+
+
+def ripe_draft_attn(h, layer, r, j, k, v, q, out, lse=None, scale=1.0, stream=None):
+    _check(lib().ripe_draft_attn(h, layer, r, j, ctypes.c_void_p(k), ctypes.c_void_p(v), ctypes.c_void_p(q),
+                                 ctypes.c_void_p(out), ctypes.c_void_p(lse or 0), float(scale),
+                                 _stream(stream)), "ripe_draft_attn")
 
 
 def ripe_verify_attn_wave(h, layer, loop_of_position, q, out, lse=None, scale=1.0, stream=None):
@@ -281,6 +289,22 @@ class RipeCache:
         op = _dev(out, torch.bfloat16, shape, "out").value
         lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
         ripe_append_verify(self.handle, layer, r, B, kp, vp, qp, op, lp, scale, stream)
+        return out
+
+    def draft_attn(self, layer, r, j, k, v, q, out=None, lse=None, scale=1.0, stream=None):
+        """Draft step: write plane r of block position j (k, v [N][1][kvH][d]) and attend its
+        query q [N][1][Hq][d] over keys up to that position."""
+        import torch
+        kshape = (self.N, 1, self.kvH, self.d)
+        shape = (self.N, 1, self.Hq, self.d)
+        kp = _dev(k, torch.bfloat16, kshape, "k").value
+        vp = _dev(v, torch.bfloat16, kshape, "v").value
+        qp = _dev(q, torch.bfloat16, shape, "q").value
+        if out is None:
+            out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+        op = _dev(out, torch.bfloat16, shape, "out").value
+        lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
+        ripe_draft_attn(self.handle, layer, r, j, kp, vp, qp, op, lp, scale, stream)
         return out
 
     def verify_attn_wave(self, layer, loop_of_position, q, out=None, lse=None, scale=1.0, stream=None):

@@ -77,12 +77,13 @@ class Case:
 
     T: committed length per sequence; W: window (>= max_T means full cache);
     oracle_seqs / oracle_kvh: subsets mirrored in the oracle (all by default);
-    oracle_planes: planes whose values the oracle keeps (all by default).
+    oracle_planes: planes whose values the oracle keeps (all by default);
+    append_block=False leaves the draft block out (kept in ``blocks`` for a later append).
     """
 
     def __init__(self, N, L, Hq, kvH, d, R, T, W, B, rho=0.88, seed=0, mode=0, max_T=None,
                  independent=False, backend="numpy", oracle_seqs=None, oracle_kvh=None,
-                 oracle_planes=None, device="cuda"):
+                 oracle_planes=None, device="cuda", append_block=True):
         self.N, self.L, self.Hq, self.kvH, self.d, self.R = N, L, Hq, kvH, d, R
         self.g = Hq // kvH
         self.T = [int(t) for t in (T if hasattr(T, "__len__") else [T] * N)]
@@ -99,7 +100,7 @@ class Case:
         self.gpu = RipeCache(N, L, Hq, kvH, d, R, W, self.max_T, B, mode)
         self.orc = orc.OracleCache(len(self.oseq), L, len(self.okvh), d, R, W, self.max_T, mode,
                                    value_planes=oracle_planes)
-        self._load()
+        self._load(append_block)
 
     # -- helpers ---------------------------------------------------------------
     def _host(self, x):
@@ -117,7 +118,7 @@ class Case:
     def _sub_block(self, x):
         return np.ascontiguousarray(self._host(x)[self.oseq][:, :, self.okvh])
 
-    def _load(self):
+    def _load(self, append_block=True):
         To = [self.T[n] for n in self.oseq]
         keep = self.orc.value_planes
         blocks = []
@@ -134,7 +135,16 @@ class Case:
                 blocks.append((l, pl, kept, seq_block(k, self.T, self.B), seq_block(v, self.T, self.B)))
                 del k, v
             self.src[l].release()
-        for l, pl, kept, kb, vb in blocks:
+        self.blocks = {(l, pl): (kb, vb) for l, pl, _, kb, vb in blocks}
+        if append_block:
+            self.append_blocks()
+        torch.cuda.synchronize()
+
+    def append_blocks(self):
+        """Append every plane of every layer's draft block on both sides."""
+        keep = self.orc.value_planes
+        for (l, pl), (kb, vb) in self.blocks.items():
+            kept = keep is None or pl in keep
             self.gpu.append_block(l, pl, self._dev(kb), self._dev(vb))
             if kept:
                 self.orc.append(l, pl, self._sub_block(kb), self._sub_block(vb))

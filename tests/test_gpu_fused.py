@@ -12,10 +12,12 @@ from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("W,B,g,d", [(16, 8, 1, 96), (5, 6, 2, 64), (0, 4, 4, 128), (10 ** 6, 8, 1, 96),
-                                     (64, 8, 4, 128)])
-def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, cuda_device):
-    N, L, kvH, R, T0, steps = 3, 2, 3, 4, 90, 6
+@pytest.mark.parametrize("W,B,g,d,T0", [(16, 8, 1, 96, 90), (5, 6, 2, 64, 90), (0, 4, 4, 128, 90),
+                                        (10 ** 6, 8, 1, 96, 90), (64, 8, 4, 128, 90),
+                                        (10 ** 6, 8, 1, 64, 60), (0, 8, 2, 96, 188)])
+def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, T0, cuda_device):
+    """T0 = 60 (full cache) and 188 (deepest only) put the block's rows across a 64-row tile edge."""
+    N, L, kvH, R, steps = 3, 2, 3, 4, 6
     max_T = T0 + B * (steps + 1)
     src = PlaneSource(N, kvH, d, R, T0, 0.88, 31, backend="torch", device=cuda_device)
     caches = [RipeCache(N, L, kvH * g, kvH, d, R, W, max_T, B) for _ in range(2)]

@@ -295,3 +295,74 @@ def test_wave_rows_match_the_brute_force_at_each_rows_loop():
     o1, _ = orc.verify_wave(c, 0, [3] * B, q, g)
     o2, _ = c.verify(0, 3, q, g)
     assert np.array_equal(o1, o2)
+
+
+# ---------------------------------------------------------------- draft phase
+def _prefix_cache(N, kvH, g, d, R, W, T, B, seed, max_extra=0):
+    src = PlaneSource(N, kvH, d, R, T + B + max_extra, 0.88, seed, independent=True)
+    PK = [src.plane(r, "K") for r in range(R)]
+    PV = [src.plane(r, "V") for r in range(R)]
+    c = orc.OracleCache(N, 1, kvH, d, R, W, T + B + max_extra)
+    for pl in range(R):
+        c.load_prefix(0, pl, [T] * N, PK[pl], PV[pl])
+    return c, PK, PV, src
+
+
+@pytest.mark.parametrize("T,W,B,r,g", [(20, 3, 5, 0, 2), (20, 0, 4, 1, 1), (6, 10, 4, 2, 3), (15, 5, 6, 4, 1)])
+def test_draft_steps_match_the_brute_force(T, W, B, r, g):
+    """Draft step j (one query at p = T + j, the drafts 0..j at plane r) equals row j of the
+    independent brute-force formulation over the same planes; the drafted rows then verified
+    as a block give the same rows."""
+    N, kvH, d, R = 1, 2, 8, 5
+    c, PK, PV, src = _prefix_cache(N, kvH, g, d, R, W, T, B, seed=17)
+    Kall = np.stack([_f64(PK[pl][0]) for pl in range(R)])
+    Vall = np.stack([_f64(PV[pl][0]) for pl in range(R)])
+    kb, vb = block_from_planes(PK[r], T, B), block_from_planes(PV[r], T, B)
+    q = src.queries(r, B, kvH * g)
+    drafts = []
+    for j in range(B):
+        out, lse = c.draft(0, r, j, kb[:, j:j + 1], vb[:, j:j + 1], q[:, j:j + 1], g, 1.2)
+        bo, bl = orc.brute_verify(Kall, Vall, T, j + 1, r, W, g, _f64(q[0, : j + 1]), 1.2)
+        assert np.abs(out[0, 0] - bo[j]).max() < 1e-12
+        assert np.abs(lse[0, 0] - bl[j]).max() < 1e-12
+        if 0 < W < T and j >= 1 and r != R - 1:
+            # planted mistake: the window measured from the cache end instead of the query
+            bc, _ = orc.brute_verify(Kall, Vall, T, j + 1, r, W, g, _f64(q[0, : j + 1]), 1.2, orc.CACHE_RELATIVE)
+            assert np.abs(out[0, 0] - bc[j]).max() > 1e-6
+        drafts.append(out[0, 0])
+    for pl in range(R):
+        c.append(0, pl, block_from_planes(PK[pl], T, B), block_from_planes(PV[pl], T, B))
+    vo, _ = c.verify(0, r, q, g, 1.2)
+    for j in range(B):
+        assert np.abs(vo[0, j] - drafts[j]).max() < 1e-12
+
+
+def test_draft_state_rules():
+    """Drafts are written in order per plane; redrafting makes later drafts stale; a
+    verification block ends the draft phase; commit discards drafts past the block."""
+    N, kvH, g, d, R, W, T, B = 1, 1, 1, 4, 3, 2, 8, 4
+    c, PK, PV, src = _prefix_cache(N, kvH, g, d, R, W, T, B, seed=19, max_extra=2)
+    kb, vb = block_from_planes(PK[0], T, B + 2), block_from_planes(PV[0], T, B + 2)
+    q = src.queries(0, B + 2, kvH * g)
+    step = lambda j: c.draft(0, 0, j, kb[:, j:j + 1], vb[:, j:j + 1], q[:, j:j + 1], g)
+    with pytest.raises(RuntimeError):
+        step(1)                                    # position 0 not drafted yet
+    for j in range(B + 2):
+        step(j)
+    assert c.present[0, 0, 0, T:T + B + 2].all()
+    step(2)                                        # redraft: positions 3.. of plane 0 are stale
+    assert c.present[0, 0, 0, T:T + 3].all() and not c.present[0, 0, 0, T + 3:].any()
+    with pytest.raises(RuntimeError):
+        step(4)
+    with pytest.raises(RuntimeError):
+        c.load_prefix(0, 0, [T], PK[0], PV[0])     # a draft is in flight
+    step(3)
+    step(4)
+    for pl in range(R):
+        c.append(0, pl, block_from_planes(PK[pl], T, 2), block_from_planes(PV[pl], T, 2))
+    with pytest.raises(RuntimeError):
+        step(0)                                    # the verification block ended the draft phase
+    c.commit([1])
+    assert int(c.T[0]) == T + 1
+    assert not c.present[0, :, 0, T + 1:].any()    # rejected block rows and drafts past the block
+    assert c.drafted.sum() == 0
