@@ -473,6 +473,46 @@ def e2e_steps(wl, args, dist_on):
                 h2d_bytes_per_step=h2d, d2h_bytes_per_step=ho.numel() * 2)
 
 
+def fixed_memory(cfg, args, device):
+    """Throughput at a fixed KV-memory budget: the largest batch of each layout whose cache fits in
+    args.fixed_memory_gb, its verification step measured at that batch and at batch 1, and the
+    two-point cost model t_step(N) = a + b * N.  Attention only: per-step costs outside this path
+    (weights) are not in a, which is why the gain at fixed memory here is the batch ratio's effect
+    on a only."""
+    import torch
+    from self_speculative_decode_b200.ripe import RipeCache
+    budget = args.fixed_memory_gb * 1e9
+    total_steps = args.warmup + 2 * args.steps + 2
+    max_T = cfg["T"] + cfg["B"] * (total_steps + 4)
+    out = {}
+    for layout in ("full", "ripe", "deepest"):
+        W = {"ripe": cfg["W"], "full": max_T, "deepest": 0}[layout]
+        probe = RipeCache(1, cfg["L"], cfg["Hq"], cfg["kvH"], cfg["d"], cfg["R"], W, max_T, cfg["B"])
+        per_seq = probe.stats()["kv_bytes"]
+        probe.close()
+        n_max = int(min(budget // per_seq, 1024))
+        res = {"kv_bytes_per_sequence": per_seq, "batch": n_max, "kv_gb": n_max * per_seq / 1e9}
+        if n_max < 1:
+            out[layout] = res
+            continue
+        for tag, n in (("n1", 1), ("nmax", n_max)):
+            r = bench_layout(dict(cfg, N=n), layout, args, args.seed, device, False, want_extras=False)
+            res[tag] = {k: r[k] for k in ("ms_per_step", "gbs", "verified_tokens_per_s", "accepted_tokens_per_s")}
+            torch.cuda.empty_cache()
+        t1, tn = res["n1"]["ms_per_step"], res["nmax"]["ms_per_step"]
+        b = (tn - t1) / (n_max - 1) if n_max > 1 else 0.0
+        res["cost_model_ms"] = {"a": t1 - b, "b_per_sequence": b}
+        out[layout] = res
+    full = out["full"].get("nmax", {}).get("verified_tokens_per_s")
+    for layout, res in out.items():
+        if full and "nmax" in res:
+            res["throughput_over_full"] = res["nmax"]["verified_tokens_per_s"] / full
+    print(json.dumps({"fixed_memory_gb": args.fixed_memory_gb, "workload": cfg["workload"],
+                      "steps": args.steps, "warmup": args.warmup, "layouts": out,
+                      "note": "largest batch whose KV cache fits the budget, verification steps timed as "
+                              "in the main benchmark (CUDA graph, CUDA events); attention only"}), flush=True)
+
+
 def profile_calls(cfg, args, device):
     """A few verify calls of one layer of the workload, nothing else: the launch ncu captures."""
     import torch
@@ -564,6 +604,8 @@ def main():
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="only run this many verify calls of layer 0 (for ncu captures) and exit")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--fixed-memory-gb", type=float, default=0.0,
+                    help="only run the fixed-memory throughput comparison at this KV budget and exit")
     ap.add_argument("--append", default="separate", choices=["separate", "fused"],
                     help="block append as its own launch before each verify, or inside it (ripe_append_verify)")
     ap.add_argument("--seed", type=int, default=0)
@@ -594,6 +636,9 @@ def main():
 
     if args.profile_calls:
         profile_calls(cfg, args, device)
+        return
+    if args.fixed_memory_gb:
+        fixed_memory(cfg, args, device)
         return
     if args.layouts is None:
         # the full cache of the long-context config needs R * T * 4 layers (137 GB): not by default

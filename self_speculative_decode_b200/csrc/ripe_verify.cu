@@ -848,14 +848,22 @@ constexpr auto ripe_verify_kernel_of() { return I::kernel; }
 // query-side configuration by the number of query rows per kv head (B * group)
 //   <= 8  : one 8-query tile per warp, 2 tile groups of 4 warps
 //   <= 16 : two 8-query tiles per warp, 2 tile groups of 4 warps
-//   <= 32 : two row groups x 4 key groups
+//   <= 32 : two row groups x 2 key groups, 2 tile groups (measured on the long-context GQA call:
+//           181 us vs 196-199 us for one tile group of 2 x 4 warps, whose 32 KB stages fit only 3 deep)
 //   <= 64 : four row groups x 2 key groups (32 keys per warp per tile)
 #ifndef RIPE_Q8_WK
 #define RIPE_Q8_WK 4
 #define RIPE_Q8_TG 2
 #endif
+#ifndef RIPE_Q32_NQT
+#define RIPE_Q32_NQT 2
+#define RIPE_Q32_WR 2
+#define RIPE_Q32_WK 2
+#define RIPE_Q32_TG 2
+#endif
+#define RIPE_Q32_CFG RIPE_Q32_NQT, RIPE_Q32_WR, RIPE_Q32_WK, RIPE_Q32_TG
 #define RIPE_QCFG_LIST(D)                                                          \
-    Inst<D, 1, 1, RIPE_Q8_WK, RIPE_Q8_TG>, Inst<D, 2, 1, 4, 2>, Inst<D, 2, 2, 4, 1>, Inst<D, 2, 4, 2, 1>
+    Inst<D, 1, 1, RIPE_Q8_WK, RIPE_Q8_TG>, Inst<D, 2, 1, 4, 2>, Inst<D, RIPE_Q32_CFG>, Inst<D, 2, 4, 2, 1>
 
 static int qcfg_of(int Mq) { return Mq <= 8 ? 0 : Mq <= 16 ? 1 : Mq <= 32 ? 2 : 3; }
 
