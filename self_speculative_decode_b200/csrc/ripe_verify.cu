@@ -48,6 +48,9 @@ struct VerifyArgs {
     // queries: block positions j0 .. j0 + qB - 1 (q, out, lse and the fused block hold qB rows
     // per sequence); a verification has j0 = 0, qB = B, a draft step j0 = its position, qB = 1
     int j0, qB;
+    // launched as clusters of 2 CTAs: when each (sequence, kv head) is split into two pieces, the
+    // CTA holding the second piece sends its partial to the first through distributed shared memory
+    int xpair;
     int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
     float scale_log2;
     // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
@@ -85,7 +88,10 @@ struct VCfg {
     static constexpr int STAGE_BYTES = 2 * NBOX * kBoxBytes;
     static constexpr int DP = D + 4;               // merge-buffer row stride (no bank conflicts)
     static constexpr int MERGE_FLOATS = NCW * NQ * DP;
-    static constexpr int MLF = NCW * NQ * 2 + ROWS * (TG * WK + 2);
+    // receive buffer of the cluster-pair merge: the partner's o [ROWS][D] and (m, l) [ROWS][2]
+    static constexpr bool XPAIR = ROWS <= 16;
+    static constexpr int XF = XPAIR ? ROWS * D + 2 * ROWS : 0;
+    static constexpr int MLF = NCW * NQ * 2 + ROWS * (TG * WK + 2) + XF;
     static constexpr int MISC = 1024 /*align*/ + 1024 /*bars, descriptors, flags*/;
     static constexpr int AVAIL = kSmemLimit - MISC - 4 * (MERGE_FLOATS + MLF) - 4 * (2 * kMaxBatch + 2);
     static constexpr int CAP = (D == 128 && TG == 1) ? RIPE_MAX_STAGES_WIDE : RIPE_MAX_STAGES;
@@ -211,6 +217,8 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     float *mml = mo + C::MERGE_FLOATS;                                   // [NCW][NQ][2]
     float *wq = mml + C::NCW * C::NQ * 2;                                // [ROWS][TG*WK] weights
     float *fin = wq + C::ROWS * TG * WK;                                 // [ROWS][2] final M, L
+    float *xo = fin + C::ROWS * 2;                                       // [ROWS][D] partner's o (XPAIR)
+    float *xml = xo + C::ROWS * D;                                       // [ROWS][2] partner's m, l
     uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);         // full[NS], empty[NS], block
     TileDesc *sdesc = reinterpret_cast<TileDesc *>(bars + 2 * NS + 2);   // [NS]
     int *sflag = reinterpret_cast<int *>(sdesc + NS);                    // [16]
@@ -239,8 +247,11 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             mbar_init(smem_addr(&bars[NS + s]), C::GW);
         }
         if (FUSED) mbar_init(smem_addr(&bars[2 * NS]), 1);  // draft block written into the ring
+        if (C::XPAIR && a.xpair) mbar_init(smem_addr(&bars[2 * NS + 1]), 1);  // partner's partial received
         mbar_fence_init();
     }
+    // the partner may arrive on this CTA's barrier: both CTAs of the pair initialise theirs first
+    if (C::XPAIR && a.xpair) cluster_sync_all();
     // rows past a short box are never written by TMA: keep them finite
     if (pa.deep_box < kTileRows || pa.ring_box < kTileRows) {
         uint4 *z = reinterpret_cast<uint4 *>(stages);
@@ -571,6 +582,61 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             fin[i * 2 + 1] = L;
         }
         named_bar_sync(1, nct);
+        if (C::XPAIR && a.xpair && pieces == 2 && !sole) {
+            // a pair of CTAs holds this (sequence, kv head): the second sends its partial into
+            // the first's shared memory, the first merges both and writes out / lse
+            const uint32_t xbar = smem_addr(&bars[2 * NS + 1]);
+            if (blockIdx.x & 1) {
+                const uint32_t rxo = mapa_shared(smem_addr(xo), 0), rxml = mapa_shared(smem_addr(xml), 0);
+                for (int e = tid; e < a.Mq * D && !abort_now; e += nct) {
+                    const int i = e / D, col = e - i * D;
+                    const int rgi = i / C::NQ, q = i - rgi * C::NQ;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int t2 = 0; t2 < TG; ++t2)
+#pragma unroll
+                        for (int k = 0; k < WK; ++k) {
+                            const float w = wq[i * (TG * WK) + t2 * WK + k];
+                            if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
+                        }
+                    st_cluster_f32(rxo + 4u * static_cast<uint32_t>(e), acc);
+                    if (col == 0) {
+                        st_cluster_f32(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2]);
+                        st_cluster_f32(rxml + 8u * static_cast<uint32_t>(i) + 4u, fin[i * 2 + 1]);
+                    }
+                }
+                fence_acq_rel_cluster();
+                named_bar_sync(1, nct);
+                if (tid == 0) mbar_arrive_remote(mapa_shared(xbar, 0));
+            } else {
+                // bounded: the partner always arrives, aborted or not
+                const bool got = mbar_wait_cluster_bounded(xbar, 0);
+                if (!got && tid == 0) atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
+                for (int e = tid; e < a.Mq * D && got && !abort_now; e += nct) {
+                    const int i = e / D, col = e - i * D;
+                    const int rgi = i / C::NQ, q = i - rgi * C::NQ;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int t2 = 0; t2 < TG; ++t2)
+#pragma unroll
+                        for (int k = 0; k < WK; ++k) {
+                            const float w = wq[i * (TG * WK) + t2 * WK + k];
+                            if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
+                        }
+                    const float M0 = fin[i * 2], M1 = xml[i * 2];
+                    const float M = fmaxf(M0, M1);
+                    const float w0 = (M0 == -INFINITY) ? 0.f : exp2f(M0 - M);
+                    const float w1 = (M1 == -INFINITY) ? 0.f : exp2f(M1 - M);
+                    const float L = w0 * fin[i * 2 + 1] + w1 * xml[i * 2 + 1];
+                    const int j = i / a.g, h = kh * a.g + (i - j * a.g);
+                    const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
+                    a.out[orow * D + col] = __float2bfloat16_rn((w0 * acc + w1 * xo[e]) / L);
+                    if (col == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
+                }
+                named_bar_sync(1, nct);
+            }
+            return;
+        }
         const int rows = sole ? a.Mq : C::ROWS;
         for (int e = tid; e < rows * D && !abort_now; e += nct) {
             const int i = e / D, col = e - i * D;
@@ -834,11 +900,40 @@ struct Inst {
             e = cudaFuncSetAttribute(kernel_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         return e;
     }
-    static void launch(const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
+    // 2 x the clusters of two CTAs that fit at once (0: no cluster launch), per instance and
+    // shared-memory size
+    static int pair_grid(bool fused, int smem, int num_sms) {
+        static int cached_smem[2] = {-1, -1}, cached[2] = {0, 0};
+        const int f = fused ? 1 : 0;
+        if (cached_smem[f] != smem) {
+            const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::THREADS + 32 * f), smem, 2,
+                                              num_sms & ~1);
+            cached[f] = 2 * n;
+            cached_smem[f] = smem;
+        }
+        return cached[f];
+    }
+    static void launch(const ripe_cache *c, int grid, const VerifyArgs &args, cudaStream_t s) {
         if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
-        const bool fused = a.blk_k != nullptr;
-        launch_pdl(fused ? kernel_fused : kernel, dim3(grid), dim3(C::THREADS + (fused ? 32 : 0)),
-                   smem_bytes_for<C>(c->N), s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
+        const bool fused = args.blk_k != nullptr;
+        auto kern = fused ? kernel_fused : kernel;
+        const dim3 block(C::THREADS + (fused ? 32 : 0));
+        const int smem = smem_bytes_for<C>(c->N);
+        VerifyArgs a = args;
+        a.xpair = 0;
+#ifndef RIPE_NO_XPAIR
+        if (C::XPAIR) {
+            const int pg = pair_grid(fused, smem, c->num_sms);
+            if (pg >= 2) {
+                int g2 = (grid + 1) & ~1;
+                if (g2 > pg) g2 = pg;
+                a.xpair = 1;
+                launch_pdl_cluster(kern, dim3(g2), block, smem, s, 2, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
+                return;
+            }
+        }
+#endif
+        launch_pdl(kern, dim3(grid), block, smem, s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
     }
 };
 
@@ -930,6 +1025,7 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.blk_k = a.blk_v = nullptr;
     a.ring_k = a.ring_v = nullptr;
     a.max_T = 0;
+    a.xpair = 0;
     a.q = static_cast<const __nv_bfloat16 *>(rv.q);
     a.out = static_cast<__nv_bfloat16 *>(rv.out);
     a.lse = rv.lse;
