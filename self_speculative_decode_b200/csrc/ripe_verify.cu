@@ -132,6 +132,35 @@ __device__ __forceinline__ int pair_of(const int *cum, int N, int kvH, int gt) {
     return n * kvH + (gt - cum[n]) / tot;
 }
 
+// How a launch of `grid` CTAs cuts `total` tiles (tot0 per (sequence, kv head) when `same`):
+// contiguous chunks of `chunk` tiles (pieces = 0), or, when several CTAs share each head,
+// `pieces` equal pieces of every head, CTA c taking piece c % pieces of head c / pieces.
+// Cuts fall on head boundaries when that costs at most kSwitchTiles tiles per CTA: a CTA then
+// never switches to another head mid-stream.
+__device__ __forceinline__ void choose_chunk(int total, int tot0, bool same, int grid, int N, int kvH, int min_chunk,
+                                             int &chunk, int &pieces) {
+    int ch = cdiv(total, grid);
+    if (ch < min_chunk) ch = min_chunk;
+    pieces = 0;
+    if (same) {
+        if (ch < tot0) {
+            int P = grid / (N * kvH);
+            if (P > tot0 / min_chunk) P = tot0 / min_chunk;
+            if (P >= 1) {
+                const int ca = cdiv(tot0, P);
+                if (ca <= ch + kSwitchTiles) {
+                    ch = ca;
+                    pieces = P;
+                }
+            }
+        } else {
+            const int ca = cdiv(ch, tot0) * tot0;
+            if (ca <= ch + kSwitchTiles) ch = ca;
+        }
+    }
+    chunk = ch;
+}
+
 // Ring tile (index within the pair's list) holding position pos of the single-loop ring [D, T + B).
 __device__ __forceinline__ int ring_tile_of(const SeqGeom &sg, const PlanArgs &pa, int pos) {
     const int o = pos - sg.D;
@@ -259,80 +288,81 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     }
     // ---- per-sequence tile counts and their prefix sums (T is written by earlier kernels)
     pdl_wait();
-    for (int n = tid; n < N; n += blockDim.x) {
-        const int T = a.T[n];
-        Ts[n] = T;
-        cum[n + 1] = seq_geom(T, pa).total * kvH;
-    }
-    if (tid == 0) cum[0] = 0;
-    __syncthreads();
-    if (warp == 0) {  // inclusive scan of cum[1..N] in chunks of 32
-        int carry = 0;
-        for (int b = 0; b < N; b += 32) {
-            int v = (b + lane < N) ? cum[b + lane + 1] : 0;
+    int total, chunk, pieces;  // pieces 0: contiguous chunks of the whole tile list
+    int tot_head = 0;          // tiles per (sequence, kv head) in piece mode
+    SeqGeom sg1 = {};          // the sequence's geometry when N == 1
+    if (N == 1) {
+        // one sequence: every thread reads T and cuts the list itself (no scan, no broadcast)
+        const int T = a.T[0];
+        sg1 = seq_geom(T, pa);
+        const int tot0 = sg1.total;
+        tot_head = tot0;
+        total = tot0 * kvH;
+        choose_chunk(total, tot0, true, static_cast<int>(gridDim.x), 1, kvH, a.min_chunk, chunk, pieces);
+        if (tid == 0) {
+            Ts[0] = T;
+            cum[0] = 0;
+            cum[1] = total;
+        }
+        __syncthreads();
+        pdl_trigger();  // the next kernel may be scheduled; it waits for this one to finish
+    } else {
+        for (int n = tid; n < N; n += blockDim.x) {
+            const int T = a.T[n];
+            Ts[n] = T;
+            cum[n + 1] = seq_geom(T, pa).total * kvH;
+        }
+        if (tid == 0) cum[0] = 0;
+        __syncthreads();
+        if (warp == 0) {  // inclusive scan of cum[1..N] in chunks of 32
+            int carry = 0;
+            for (int b = 0; b < N; b += 32) {
+                int v = (b + lane < N) ? cum[b + lane + 1] : 0;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int u = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += u;
-            }
-            if (b + lane < N) cum[b + lane + 1] = v + carry;
-            carry += __shfl_sync(0xffffffffu, v, 31);
-        }
-    }
-    __syncthreads();
-
-    pdl_trigger();  // the next kernel may be scheduled; it waits for this one to finish
-    const int total = cum[N];
-    if (warp == 0) {
-        // equal tile counts for every (sequence, kv head)?
-        const int tot0 = cum[1] / kvH;
-        bool same = true;
-        for (int b = 0; b < N; b += 32) {
-            const bool ok = (b + lane >= N) || (cum[b + lane + 1] - cum[b + lane] == cum[1]);
-            same = same && __all_sync(0xffffffffu, ok);
-        }
-        if (lane == 0) {
-            int ch = cdiv(total, static_cast<int>(gridDim.x));
-            if (ch < a.min_chunk) ch = a.min_chunk;
-            int pieces = 0;
-            if (same) {
-                // cut at (sequence, kv head) boundaries when that costs at most kSwitchTiles
-                // tiles per CTA: a CTA then never switches to another head mid-stream
-                if (ch < tot0) {
-                    // several CTAs per head: `pieces` equal pieces of each head, CTA c taking
-                    // piece c % pieces of head c / pieces
-                    int P = static_cast<int>(gridDim.x) / (N * kvH);
-                    if (P > tot0 / a.min_chunk) P = tot0 / a.min_chunk;
-                    if (P >= 1) {
-                        const int ca = cdiv(tot0, P);
-                        if (ca <= ch + kSwitchTiles) {
-                            ch = ca;
-                            pieces = P;
-                        }
-                    }
-                } else {
-                    const int ca = cdiv(ch, tot0) * tot0;
-                    if (ca <= ch + kSwitchTiles) ch = ca;
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += u;
                 }
+                if (b + lane < N) cum[b + lane + 1] = v + carry;
+                carry += __shfl_sync(0xffffffffu, v, 31);
             }
-            sflag[6] = ch;
-            sflag[7] = pieces;
         }
+        __syncthreads();
+        pdl_trigger();
+        total = cum[N];
+        if (warp == 0) {
+            // equal tile counts for every (sequence, kv head)?
+            bool same = true;
+            for (int b = 0; b < N; b += 32) {
+                const bool ok = (b + lane >= N) || (cum[b + lane + 1] - cum[b + lane] == cum[1]);
+                same = same && __all_sync(0xffffffffu, ok);
+            }
+            if (lane == 0) {
+                int ch, pc;
+                choose_chunk(total, cum[1] / kvH, same, static_cast<int>(gridDim.x), N, kvH, a.min_chunk, ch, pc);
+                sflag[6] = ch;
+                sflag[7] = pc;
+            }
+        }
+        __syncthreads();
+        chunk = sflag[6];
+        pieces = sflag[7];
+        if (pieces) tot_head = cum[1] / kvH;
     }
-    __syncthreads();
-    const int chunk = sflag[6];
-    const int pieces = sflag[7];  // 0: contiguous chunks of the whole tile list
-    int g_begin, g_end;
+    int g_begin, g_end, head = 0;
     if (pieces) {
-        const int tot0 = cum[1] / kvH, h = blockIdx.x / pieces;
-        g_begin = h * tot0 + (blockIdx.x - h * pieces) * chunk;
-        g_end = min(min(g_begin + chunk, (h + 1) * tot0), total);
+        head = blockIdx.x / pieces;
+        g_begin = head * tot_head + (blockIdx.x - head * pieces) * chunk;
+        g_end = min(min(g_begin + chunk, (head + 1) * tot_head), total);
     } else {
         g_begin = blockIdx.x * chunk;
         g_end = min(total, g_begin + chunk);
     }
     if (g_begin >= g_end) return;
     const int ntiles = g_end - g_begin;
+    // (sequence, kv head) pairs of this CTA's first and last tiles
+    const int P_first = pieces ? head : pair_of(cum, N, kvH, g_begin);
+    const int P_last = pieces ? head : pair_of(cum, N, kvH, g_end - 1);
 
     const uint32_t full0 = smem_addr(&bars[0]);
     const uint32_t empty0 = smem_addr(&bars[NS]);
@@ -355,12 +385,21 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     if (warp == C::NCW) {
         // ================================================================ producer (one thread)
         if (lane == 0) {
-            int n = seq_of(cum, N, g_begin);
-            SeqGeom sg = seq_geom(Ts[n], pa);
-            int rel = g_begin - cum[n];
-            int kh = rel / sg.total;
-            int lt = rel - kh * sg.total;
-            const int P0 = n * kvH + kh;
+            int n, kh, lt;
+            SeqGeom sg;
+            if (pieces) {  // one head per CTA: no search, no division by the head's tile count
+                n = N == 1 ? 0 : P_first / kvH;
+                kh = P_first - n * kvH;
+                sg = N == 1 ? sg1 : seq_geom(Ts[n], pa);
+                lt = (blockIdx.x - head * pieces) * chunk;
+            } else {
+                n = seq_of(cum, N, g_begin);
+                sg = seq_geom(Ts[n], pa);
+                const int rel = g_begin - cum[n];
+                kh = rel / sg.total;
+                lt = rel - kh * sg.total;
+            }
+            const int P0 = P_first;
             int i = 0;
             bool ok = true;
             // with a fused append, the tiles holding the rows this launch writes wait until the
@@ -402,7 +441,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     }
                 }
                 if (i == NS - 1) {  // pipeline full: warm L2 with the query rows of the later pairs
-                    const int p_last = pair_of(cum, N, kvH, g_end - 1);
+                    const int p_last = P_last;
                     for (int p = P0 + 1; p <= p_last; ++p) {
                         const int pn = p / kvH, pk = p - pn * kvH;
                         for (int j = 0; j < a.qB; ++j) {
@@ -464,8 +503,6 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     float m_ref[NQT][2], l_run[NQT][2];
     uint32_t qb[D / 16][NQT][2];
 
-    const int P_first = pair_of(cum, N, kvH, g_begin);
-    const int P_last = pair_of(cum, N, kvH, g_end - 1);
     int fin_next = P_first;  // next pair to finalize (every consumer warp finalizes each pair once)
     int st_pair = -1;        // pair whose partial state this warp holds
     bool aborted = false;
@@ -582,28 +619,36 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             fin[i * 2 + 1] = L;
         }
         named_bar_sync(1, nct);
+        // four consecutive columns of one row per thread: float4 shared-memory reads (the
+        // row's weights are read once), 16-byte stores
+        auto row_acc = [&](int i, int c0) {
+            const int rgi = i / C::NQ, q = i - rgi * C::NQ;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int t2 = 0; t2 < TG; ++t2)
+#pragma unroll
+                for (int k = 0; k < WK; ++k) {
+                    const float w = wq[i * (TG * WK) + t2 * WK + k];
+                    if (w != 0.f) {
+                        const float4 v = *reinterpret_cast<const float4 *>(
+                            &mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + c0]);
+                        acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+                    }
+                }
+            return acc;
+        };
+        constexpr int D4 = D / 4;
         if (C::XPAIR && a.xpair && pieces == 2 && !sole) {
             // a pair of CTAs holds this (sequence, kv head): the second sends its partial into
             // the first's shared memory, the first merges both and writes out / lse
             const uint32_t xbar = smem_addr(&bars[2 * NS + 1]);
             if (blockIdx.x & 1) {
                 const uint32_t rxo = mapa_shared(smem_addr(xo), 0), rxml = mapa_shared(smem_addr(xml), 0);
-                for (int e = tid; e < a.Mq * D && !abort_now; e += nct) {
-                    const int i = e / D, col = e - i * D;
-                    const int rgi = i / C::NQ, q = i - rgi * C::NQ;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int t2 = 0; t2 < TG; ++t2)
-#pragma unroll
-                        for (int k = 0; k < WK; ++k) {
-                            const float w = wq[i * (TG * WK) + t2 * WK + k];
-                            if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
-                        }
-                    st_cluster_f32(rxo + 4u * static_cast<uint32_t>(e), acc);
-                    if (col == 0) {
-                        st_cluster_f32(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2]);
-                        st_cluster_f32(rxml + 8u * static_cast<uint32_t>(i) + 4u, fin[i * 2 + 1]);
-                    }
+                for (int e = tid; e < a.Mq * D4 && !abort_now; e += nct) {
+                    const int i = e / D4, c0 = 4 * (e - i * D4);
+                    const float4 acc = row_acc(i, c0);
+                    st_cluster_v4(rxo + 4u * static_cast<uint32_t>(i * D + c0), acc);
+                    if (c0 == 0) st_cluster_v2(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2], fin[i * 2 + 1]);
                 }
                 fence_acq_rel_cluster();
                 named_bar_sync(1, nct);
@@ -612,53 +657,43 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 // bounded: the partner always arrives, aborted or not
                 const bool got = mbar_wait_cluster_bounded(xbar, 0);
                 if (!got && tid == 0) atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
-                for (int e = tid; e < a.Mq * D && got && !abort_now; e += nct) {
-                    const int i = e / D, col = e - i * D;
-                    const int rgi = i / C::NQ, q = i - rgi * C::NQ;
-                    float acc = 0.f;
-#pragma unroll
-                    for (int t2 = 0; t2 < TG; ++t2)
-#pragma unroll
-                        for (int k = 0; k < WK; ++k) {
-                            const float w = wq[i * (TG * WK) + t2 * WK + k];
-                            if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
-                        }
+                for (int e = tid; e < a.Mq * D4 && got && !abort_now; e += nct) {
+                    const int i = e / D4, c0 = 4 * (e - i * D4);
+                    const float4 acc = row_acc(i, c0);
+                    const float4 o1 = *reinterpret_cast<const float4 *>(&xo[i * D + c0]);
                     const float M0 = fin[i * 2], M1 = xml[i * 2];
                     const float M = fmaxf(M0, M1);
                     const float w0 = (M0 == -INFINITY) ? 0.f : exp2f(M0 - M);
                     const float w1 = (M1 == -INFINITY) ? 0.f : exp2f(M1 - M);
                     const float L = w0 * fin[i * 2 + 1] + w1 * xml[i * 2 + 1];
+                    const float inv = 1.f / L;
                     const int j = i / a.g, h = kh * a.g + (i - j * a.g);
                     const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
-                    a.out[orow * D + col] = __float2bfloat16_rn((w0 * acc + w1 * xo[e]) / L);
-                    if (col == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
+                    __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + c0]);
+                    op[0] = __floats2bfloat162_rn((w0 * acc.x + w1 * o1.x) * inv, (w0 * acc.y + w1 * o1.y) * inv);
+                    op[1] = __floats2bfloat162_rn((w0 * acc.z + w1 * o1.z) * inv, (w0 * acc.w + w1 * o1.w) * inv);
+                    if (c0 == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
                 }
                 named_bar_sync(1, nct);
             }
             return;
         }
         const int rows = sole ? a.Mq : C::ROWS;
-        for (int e = tid; e < rows * D && !abort_now; e += nct) {
-            const int i = e / D, col = e - i * D;
-            const int rgi = i / C::NQ, q = i - rgi * C::NQ;
-            float acc = 0.f;
-#pragma unroll
-            for (int t2 = 0; t2 < TG; ++t2)
-#pragma unroll
-                for (int k = 0; k < WK; ++k) {
-                    // a warp that saw no key of this row left its slice of the buffer stale
-                    const float w = wq[i * (TG * WK) + t2 * WK + k];
-                    if (w != 0.f) acc += mo[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * C::DP + col] * w;
-                }
+        for (int e = tid; e < rows * D4 && !abort_now; e += nct) {
+            const int i = e / D4, c0 = 4 * (e - i * D4);
+            const float4 acc = row_acc(i, c0);  // a warp that saw no key of the row has weight 0
             if (sole) {
+                const float inv = 1.f / fin[i * 2 + 1];
                 const int j = i / a.g, h = kh * a.g + (i - j * a.g);
                 const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
-                a.out[orow * D + col] = __float2bfloat16_rn(acc / fin[i * 2 + 1]);
-                if (col == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
+                __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + c0]);
+                op[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+                op[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+                if (c0 == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
             } else {
                 const size_t prow = (static_cast<size_t>(blockIdx.x) + p) * C::ROWS + i;
-                a.part_o[prow * D + col] = acc;
-                if (col == 0) {
+                *reinterpret_cast<float4 *>(&a.part_o[prow * D + c0]) = acc;
+                if (c0 == 0) {
                     a.part_ml[prow * 2] = fin[i * 2];
                     a.part_ml[prow * 2 + 1] = fin[i * 2 + 1];
                 }
@@ -851,6 +886,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     };
 
     reset_state();
+    // the first pair's queries: loaded while its first tile is still in flight
+    st_pair = P_first;
+    load_q(P_first / kvH, P_first - (P_first / kvH) * kvH);
     for (int i = tg; i < ntiles; i += TG) {
         const int s = i % NS;
         if (!mbar_wait_bounded(full0 + 8 * s, (i / NS) & 1)) {
