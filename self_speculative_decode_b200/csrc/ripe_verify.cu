@@ -276,7 +276,12 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             mbar_init(smem_addr(&bars[NS + s]), C::GW);
         }
         if (FUSED) mbar_init(smem_addr(&bars[2 * NS]), 1);  // draft block written into the ring
-        if (C::XPAIR && a.xpair) mbar_init(smem_addr(&bars[2 * NS + 1]), 1);  // partner's partial received
+        if (C::XPAIR && a.xpair) {
+            // partner's partial received: the first CTA of a pair expects its bytes (used only
+            // when the pair splits one head; otherwise nothing waits on it)
+            mbar_init(smem_addr(&bars[2 * NS + 1]), 1);
+            if (!(blockIdx.x & 1)) mbar_expect_tx(smem_addr(&bars[2 * NS + 1]), a.Mq * (D * 4 + 8));
+        }
         mbar_fence_init();
     }
     // the partner may arrive on this CTA's barrier: both CTAs of the pair initialise theirs first
@@ -643,18 +648,18 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             // the first's shared memory, the first merges both and writes out / lse
             const uint32_t xbar = smem_addr(&bars[2 * NS + 1]);
             if (blockIdx.x & 1) {
+                // asynchronous stores that complete the partner's expected byte count (sent even
+                // after an abort, so that the partner never waits out its bound)
                 const uint32_t rxo = mapa_shared(smem_addr(xo), 0), rxml = mapa_shared(smem_addr(xml), 0);
-                for (int e = tid; e < a.Mq * D4 && !abort_now; e += nct) {
+                const uint32_t rbar = mapa_shared(xbar, 0);
+                for (int e = tid; e < a.Mq * D4; e += nct) {
                     const int i = e / D4, c0 = 4 * (e - i * D4);
                     const float4 acc = row_acc(i, c0);
-                    st_cluster_v4(rxo + 4u * static_cast<uint32_t>(i * D + c0), acc);
-                    if (c0 == 0) st_cluster_v2(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2], fin[i * 2 + 1]);
+                    st_async_v4(rxo + 4u * static_cast<uint32_t>(i * D + c0), acc, rbar);
+                    if (c0 == 0) st_async_v2(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2], fin[i * 2 + 1], rbar);
                 }
-                fence_acq_rel_cluster();
-                named_bar_sync(1, nct);
-                if (tid == 0) mbar_arrive_remote(mapa_shared(xbar, 0));
             } else {
-                // bounded: the partner always arrives, aborted or not
+                // bounded wait for the partner's bytes
                 const bool got = mbar_wait_cluster_bounded(xbar, 0);
                 if (!got && tid == 0) atomicOr(a.err, RIPE_DEVERR_WAIT_TIMEOUT);
                 for (int e = tid; e < a.Mq * D4 && got && !abort_now; e += nct) {
