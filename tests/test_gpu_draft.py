@@ -57,6 +57,7 @@ def _then_verify(c, layer, loops, outs, J):
     dict(N=2, Hq=3, kvH=3, d=96, R=4, T=[0, 129], W=5, B=6),           # empty prefix, ragged tail
     dict(N=2, Hq=4, kvH=1, d=64, R=3, T=[70, 64], W=0, B=4),           # deepest-only layout, g = 4
     dict(N=1, Hq=2, kvH=2, d=64, R=3, T=[200], W=10 ** 6, B=5),       # full cache
+    dict(N=2, Hq=60, kvH=30, d=96, R=4, T=[500, 500], W=16, B=8),      # two CTAs per head (cluster pairs)
 ])
 def test_draft_phase_parity(kw, cuda_device):
     c = Case(L=1, seed=21, independent=True, append_block=False, **kw)

@@ -110,3 +110,18 @@ def test_block_split_independence_on_gpu(cuda_device):
     # same keys and planes: both splits are within the parity tolerance of the exact value
     for key in a:
         assert_same_result(a[key], b[key], f"position {key[0]} loop {key[1]}")
+
+
+@pytest.mark.parametrize("kw", [
+    dict(N=2, Hq=30, kvH=30, d=96, R=4, T=[700, 700], W=64, B=8),            # 60 heads, two sequences
+    dict(N=3, Hq=48, kvH=24, d=128, R=3, T=[900, 900, 900], W=32, B=8),      # GQA 2: 16 query rows
+    dict(N=1, Hq=40, kvH=40, d=64, R=3, T=[2000], W=16, B=4),                # three CTAs per head
+])
+def test_heads_split_over_ctas(kw, cuda_device):
+    """Fewer heads than SMs with equal lengths: each head is split into equal pieces, one per CTA.
+    Two pieces are merged inside a 2-CTA cluster through shared memory; more go through global
+    scratch.  Independent planes, every loop."""
+    c = Case(L=1, seed=41, independent=True, **kw)
+    for r in range(kw["R"]):
+        c.check(0, r)
+    c.close()
