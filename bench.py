@@ -79,16 +79,26 @@ def draft_bytes(cfg, T_list, r, j, W):
     return keys * row + 2 * cfg["N"] * cfg["Hq"] * cfg["d"] * 2
 
 
+def _code_only(text):
+    """C/C++/CUDA source without comments and blank-run whitespace (comment edits do not
+    change what a capture measured)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
 def sources_digest():
-    """sha256 over the library's CUDA sources and C header (ties an ncu capture to a kernel version)."""
+    """sha256 over the code of the library's CUDA sources and C header, comments removed
+    (ties an ncu capture to a kernel version)."""
     import glob
     import hashlib
     h = hashlib.sha256()
     files = sorted(glob.glob(os.path.join(ROOT, "self_speculative_decode_b200", "csrc", "*.cu*")))
     files += [os.path.join(ROOT, "include", "ripe.h")]
     for path in files:
-        with open(path, "rb") as f:
-            h.update(os.path.basename(path).encode() + b"\0" + f.read())
+        with open(path, encoding="utf-8") as f:
+            h.update(os.path.basename(path).encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()
 
 

@@ -143,8 +143,9 @@ int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, c
  *   scale  logit scale (1/sqrt(d) for unscaled queries)
  * Requires plane r of the block appended for this layer (else RIPE_ESTATE).
  * Work: split-KV over the deepest-plane region and the window ring in one persistent
- * launch; partial results are merged in the same launch through per-call scratch owned by
- * the cache.
+ * launch; partial results are merged in the same launch, through the shared memory of a
+ * 2-CTA cluster when two CTAs share a (sequence, kv head), else through per-call scratch
+ * owned by the cache.
  */
 int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out, float *lse,
                      float scale, void *stream);

@@ -11,7 +11,9 @@
 //     at plane r, and at most two "dual" ring tiles at plane R-1 holding the window keys
 //     that later queries of the block see at the deepest plane (query-relative window).
 //     All lists are concatenated and cut into equal contiguous chunks, one per CTA, so
-//     ragged lengths and the three layouts (full, RIPE, deepest-only) balance the same way.
+//     ragged lengths and the three layouts (full, RIPE, deepest-only) balance the same way;
+//     when every head has the same tile count and there are fewer heads than CTAs, each
+//     head is cut into equal pieces instead, one per CTA, so that no CTA straddles two heads.
 //   * One producer thread streams 64-key K/V tiles with 3-D TMA loads (64-byte swizzle, no
 //     multicast) into a shared-memory ring of NS stages guarded by mbarriers, and writes a
 //     small descriptor of each tile (sequence, kv head, kind, first key, count) beside it.
@@ -23,9 +25,11 @@
 //   * Online softmax in base 2; the reference maximum only moves when a tile's maximum
 //     exceeds it by more than 8 (so probabilities stay <= 2^8), which skips most O rescales
 //     and is exact.  Full deepest-plane tiles take a path without masks.
-//   * A CTA that covers a whole (sequence, kv head) writes the output directly.  Otherwise
-//     it writes an unnormalised partial (o, m, l); the last CTA to arrive (atomic counter,
-//     no spinning) merges the partials by log-sum-exp and writes out / lse.
+//   * A CTA that covers a whole (sequence, kv head) writes the output directly.  A head cut
+//     into two pieces is held by the two CTAs of a cluster: the second sends its unnormalised
+//     partial (o, m, l) into the first's shared memory (st.async counted on an mbarrier) and
+//     the first merges the two by log-sum-exp.  Otherwise the CTAs write partials to global
+//     scratch; the last to arrive (atomic counter, no spinning) merges them.
 //   * Every wait is bounded: on timeout the kernel records RIPE_DEVERR_WAIT_TIMEOUT, drains
 //     its own copies in flight and returns without writing further results.
 #include <type_traits>
