@@ -68,6 +68,7 @@ def verify_bytes(cfg, T_list, r):
 
 
 DRAFT_LOOPS = 4  # draft depth of the timed draft phase: loops 0..3 of 32
+DRAFT_SINK, DRAFT_WINDOW = 4, 256  # windowed draft attention: attention sink and sliding window
 
 
 def draft_bytes(cfg, T_list, r, j, W):
@@ -86,6 +87,19 @@ def _code_only(text):
     text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
     text = re.sub(r"//[^\n]*", "", text)
     return "\n".join(" ".join(line.split()) for line in text.splitlines() if line.strip())
+
+
+def draft_window_bytes(cfg, T_list, r, j, W, sink, window):
+    """Bytes one windowed draft step reads: the sink and window keys of the deepest-plane
+    region, the window ring up to the query, the dual window keys, the query and the output."""
+    row = 4 * cfg["kvH"] * cfg["d"]
+    keys = 0
+    for T in T_list:
+        D = max(0, T - W)
+        se = min(sink, D)
+        dw0 = min(max(T + j - window, se), D)
+        keys += se + (D - dw0) + (T + j + 1 - D) + dual_keys(T, W, j + 1, cfg["R"], r)
+    return keys * row + 2 * cfg["N"] * cfg["Hq"] * cfg["d"] * 2
 
 
 def sources_digest():
@@ -440,16 +454,32 @@ def draft_timing(wl, args, dist_on):
                 for r in range(rd):
                     c.draft_attn(layer, r, j, dk[layer][r][j], dv[layer][r][j], dq[layer][r][j], out=dout)
     launches = c.launch_count() - n0
+    # the same phase with windowed draft attention (attention sink + sliding window)
+    gw = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw):
+        for j in range(B):
+            for layer in range(L):
+                for r in range(rd):
+                    c.draft_attn(layer, r, j, dk[layer][r][j], dv[layer][r][j], dq[layer][r][j], out=dout,
+                                 sink=DRAFT_SINK, window=DRAFT_WINDOW)
     reps = max(3, args.steps)
     g.replay()
+    gw.replay()
     ms = max_over_ranks(time_region(lambda: [g.replay() for _ in range(reps)], dist_on), dist_on)
+    msw = max_over_ranks(time_region(lambda: [gw.replay() for _ in range(reps)], dist_on), dist_on)
     T_now = c.sync_lengths()
     nbytes = sum(draft_bytes(cfg, T_now, r, j, wl.W) for j in range(B) for r in range(rd)) * L
-    phase_ms = ms / reps
+    wbytes = sum(draft_window_bytes(cfg, T_now, r, j, wl.W, DRAFT_SINK, DRAFT_WINDOW)
+                 for j in range(B) for r in range(rd)) * L
+    phase_ms, wphase_ms = ms / reps, msw / reps
     return dict(loops=rd, calls_per_block=launches, ms_per_block=phase_ms,
                 us_per_call=phase_ms * 1e3 / launches, bytes_per_call=nbytes / launches,
                 gbs=nbytes / (phase_ms * 1e-3) / 1e9,
-                drafted_tokens_per_s=cfg["N"] * B / (phase_ms * 1e-3))
+                drafted_tokens_per_s=cfg["N"] * B / (phase_ms * 1e-3),
+                windowed={"sink": DRAFT_SINK, "window": DRAFT_WINDOW, "ms_per_block": wphase_ms,
+                          "us_per_call": wphase_ms * 1e3 / launches, "bytes_per_call": wbytes / launches,
+                          "gbs": wbytes / (wphase_ms * 1e-3) / 1e9,
+                          "drafted_tokens_per_s": cfg["N"] * B / (wphase_ms * 1e-3)})
 
 
 def e2e_steps(wl, args, dist_on):

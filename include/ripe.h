@@ -181,6 +181,20 @@ int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, con
                     const void *q, void *out, float *lse, float scale, void *stream);
 
 /*
+ * ripe_draft_attn with windowed draft attention: a sliding window plus an attention sink on
+ * the draft's attention only, verification untouched ("Windowed-MTP: Removing the
+ * Full-Context Draft-KV Tax at Million-Token Context", abstract).  The query of position
+ * p = T_n + j attends only to the keys t <= p with t < sink or t >= p - window, each read at
+ * the plane the rule of ripe_verify_attn gives it; the deepest-plane keys in between are not
+ * read, so the draft's read is bounded by sink + window + W + B positions whatever T_n is.
+ *   sink    >= 0 positions at the start of the sequence always attended
+ *   window  >= 0; window >= T_n + j attends every key (the same result as ripe_draft_attn)
+ * Other arguments, state rules and errors as for ripe_draft_attn.
+ */
+int ripe_draft_attn_window(ripe_cache_t *c, int layer, int r, int j, int sink, int window, const void *k,
+                           const void *v, const void *q, void *out, float *lse, float scale, void *stream);
+
+/*
  * Verification attention with a loop per block position: block position j is evaluated
  * exactly as ripe_verify_attn(.., loop_of_position[j], ..) would evaluate it.  This is the
  * shape of a wavefront schedule, where one batched pass of the looped block holds positions

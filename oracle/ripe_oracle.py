@@ -7,7 +7,9 @@ the CUDA library and never takes an input or an expected value from it.
 Source: "Prefix Keys and Values Matter Late: RIPE Caching for Self-Speculative
 Decoding in Looped Language Models" (arXiv 2610.34436), abstract; and the
 WaveFront Decoding write-up (rit.work blog, section on drafting and checking in
-one pass) for the accept/rollback semantics.
+one pass) for the accept/rollback semantics; "Windowed-MTP: Removing the
+Full-Context Draft-KV Tax at Million-Token Context", abstract, for the windowed
+draft attention (a sliding window plus an attention sink on the draft only).
 
 Contents
   * ``verify``         verification attention of one loop, through the C oracle
@@ -25,7 +27,9 @@ Contents
   * ``OracleCache.draft``  one draft-phase step: plane r of block position j stored,
                        then the query of that position attends with the verification
                        rule for p = T + j (draft-then-verify builds the block one
-                       position at a time at a shallow loop).
+                       position at a time at a shallow loop); optionally windowed.
+  * ``windowed_draft`` draft attention restricted to an attention sink and a sliding
+                       window (the Windowed-MTP abstract), planes by the RIPE rule.
 Every function here is pinned by ``tests/test_oracle_*.py``; none is "parity
 unpinned".
 """
@@ -257,7 +261,7 @@ class OracleCache:
         self.drafted[:] = 0
 
     # -- draft phase --------------------------------------------------------------
-    def draft(self, layer, r, j, k, v, q_bits, g, scale=1.0):
+    def draft(self, layer, r, j, k, v, q_bits, g, scale=1.0, sink=None, window=None):
         """Draft step at loop r for block position j of every sequence.
 
         Stores plane r of position T_n + j (k, v bits [N][1][kvH][d]); positions after j of
@@ -265,6 +269,11 @@ class OracleCache:
         attends over keys t <= p: the definition of ``verify`` with a block of j + 1
         positions, row j (the drafts 0 .. j at plane r, the window from p, older keys at the
         deepest plane).  Returns (out [N][1][Hq][d], lse [N][1][Hq]) in fp64.
+
+        With ``sink`` and ``window`` (windowed draft attention: a sliding window plus an
+        attention sink on the draft's attention only, the Windowed-MTP abstract), only the
+        keys t < sink and t >= p - window are attended, each at the plane the rule above
+        gives it (``windowed_draft``).
         """
         if self.B:
             raise RuntimeError("draft step with a verification block in flight")
@@ -288,6 +297,10 @@ class OracleCache:
             raise RuntimeError("a draft step needs the values of planes r and R-1")
         Kr, Vr, Kl, Vl, _ = self.verify_inputs(layer, r)
         qb = bf16_to_f64(q_bits)
+        if sink is not None or window is not None:
+            return windowed_draft(self.T, j, r, self.R, self.W, g, Kr, Vr, Kl, Vl, qb[:, 0],
+                                  0 if sink is None else int(sink),
+                                  int(self.max_T) if window is None else int(window), scale, self.mode)
         qfull = np.zeros((self.N, j + 1) + qb.shape[2:])
         qfull[:, j] = qb[:, 0]
         out, lse = verify(self.T, j + 1, r, self.R, self.W, g, Kr, Vr, Kl, Vl, qfull, scale, self.mode)
@@ -319,6 +332,41 @@ class OracleCache:
         Kr, Vr, Kl, Vl, _ = self.verify_inputs(layer, r)
         return verify(self.T, self.B, r, self.R, self.W, g, Kr, Vr, Kl, Vl,
                       bf16_to_f64(q_bits), scale, self.mode)
+
+
+def windowed_draft(T, j, r, R, W, g, Kr, Vr, Kl, Vl, q, sink, window, scale=1.0, mode=QUERY_RELATIVE):
+    """Windowed draft attention of one query per sequence (numpy, fp64).
+
+    The query of position p = T_n + j attends over the keys t <= p with t < sink (the
+    attention sink) or t >= p - window (the sliding window), each read at the plane the RIPE
+    rule gives it (``plane_of``): plane r for the draft rows t >= T_n and the RIPE window,
+    plane R-1 otherwise.  Kr/Vr/Kl/Vl as for ``verify`` (NaN where nothing is stored);
+    q [N][Hq][d].  Returns (out [N][1][Hq][d], lse [N][1][Hq]).
+    """
+    T = np.asarray(T, dtype=np.int64)
+    N, kvH, _, d = Kr.shape
+    Hq = q.shape[1]
+    out = np.zeros((N, 1, Hq, d))
+    lse = np.zeros((N, 1, Hq))
+    for n in range(N):
+        Tn = int(T[n])
+        p = Tn + j
+        keys = [t for t in range(p + 1) if t < sink or t >= p - window]
+        planes = np.array([plane_of(p, t, r, R, Tn, W, mode) for t in keys])
+        idx = np.array(keys)
+        deep = planes == R - 1
+        for h in range(Hq):
+            kh = h // g
+            K = np.where(deep[:, None], Kl[n, kh, idx], Kr[n, kh, idx])
+            V = np.where(deep[:, None], Vl[n, kh, idx], Vr[n, kh, idx])
+            if np.isnan(K).any() or np.isnan(V).any():
+                raise RuntimeError("oracle read a plane that the cache does not store")
+            s = scale * (K @ q[n, h])
+            m = s.max()
+            e = np.exp(s - m)
+            out[n, 0, h] = (e[:, None] * V).sum(0) / e.sum()
+            lse[n, 0, h] = m + np.log(e.sum())
+    return out, lse
 
 
 def verify_wave(cache, layer, loop_of_position, q_bits, g, scale=1.0):

@@ -263,8 +263,8 @@ int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, 
     return RIPE_OK;
 }
 
-int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, const void *v, const void *q,
-                    void *out, float *lse, float scale, void *stream) {
+static int draft_step(ripe_cache_t *c, int layer, int r, int j, int sink, int window, const void *k, const void *v,
+                      const void *q, void *out, float *lse, float scale, void *stream) {
     if (!c || !k || !v || !q || !out || layer < 0 || layer >= c->L || r < 0 || r >= c->R || j < 0 ||
         j >= c->max_B)
         return RIPE_EINVAL;
@@ -274,11 +274,23 @@ int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, con
         if (c->T[n] + j + 1 > c->max_T) return RIPE_ECAPACITY;
     DeviceGuard g(c->device);
     if (!g.ok) return RIPE_ECUDA;
-    const int st = launch_draft(c, layer, r, j, k, v, q, out, lse, scale, static_cast<cudaStream_t>(stream));
+    const int st = launch_draft(c, layer, r, j, k, v, q, out, lse, scale, static_cast<cudaStream_t>(stream), sink,
+                                window);
     if (st != RIPE_OK) return st;
     c->drafted[idx] = j + 1;  // a later position of this plane is stale once j is redrafted
     c->prefix_set = true;
     return RIPE_OK;
+}
+
+int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, const void *v, const void *q,
+                    void *out, float *lse, float scale, void *stream) {
+    return draft_step(c, layer, r, j, 0, -1, k, v, q, out, lse, scale, stream);
+}
+
+int ripe_draft_attn_window(ripe_cache_t *c, int layer, int r, int j, int sink, int window, const void *k,
+                           const void *v, const void *q, void *out, float *lse, float scale, void *stream) {
+    if (sink < 0 || window < 0) return RIPE_EINVAL;
+    return draft_step(c, layer, r, j, sink, window, k, v, q, out, lse, scale, stream);
 }
 
 int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q, void *out,

@@ -72,6 +72,9 @@ enum TileKind { kDeep = 0, kRing = 1, kDual = 2 };
 
 struct PlanArgs {
     int W, B, R, ring_slots, deep_box, ring_box, mode_eff;
+    // windowed draft attention (dwin >= 0): the query of block position dj attends only to keys
+    // t < sink and t >= T + dj - dwin; the deepest-plane tiles in between are not read
+    int sink, dwin, dj;
     int nloops;                      // distinct loops of this call (1 for a single-loop verify)
     uint8_t loop[kMaxQueryRows];     // those loops; the ring is read once per loop
     uint8_t jloop[kMaxQueryRows];    // loop of each block position j
@@ -79,6 +82,7 @@ struct PlanArgs {
 
 struct SeqGeom {
     int T, D, nd, s0;  // s0: ring slot of position D
+    int se, nds, dw0;  // windowed draft: sink keys [0, se) in nds tiles, then deep keys [dw0, D)
     int ring_len, ring_first, nr1, nr;
     int dual_len, dual_first, ndl1, ndl;
     int total;
@@ -99,7 +103,16 @@ __host__ __device__ __forceinline__ SeqGeom seq_geom(int T, const PlanArgs &a) {
     SeqGeom s;
     s.T = T;
     s.D = T - a.W > 0 ? T - a.W : 0;
-    s.nd = ctiles(s.D, a.deep_box);
+    if (a.dwin >= 0) {
+        s.se = a.sink < s.D ? a.sink : s.D;
+        s.nds = ctiles(s.se, a.deep_box);
+        const int ws = T + a.dj - a.dwin;
+        s.dw0 = ws > s.se ? (ws < s.D ? ws : s.D) : s.se;
+        s.nd = s.nds + ctiles(s.D - s.dw0, a.deep_box);
+    } else {
+        s.se = s.nds = s.dw0 = 0;
+        s.nd = ctiles(s.D, a.deep_box);
+    }
     s.s0 = s.D % a.ring_slots;
     s.ring_len = T + a.B - s.D;
     s.ring_first = s.ring_len < a.ring_slots - s.s0 ? s.ring_len : a.ring_slots - s.s0;
@@ -122,8 +135,15 @@ __host__ __device__ __forceinline__ Tile tile_at(const SeqGeom &s, int lt, const
     Tile t;
     if (lt < s.nd) {
         t.kind = kDeep;
-        t.t0 = lt * a.deep_box;
-        t.cnt = (s.D - t.t0) < a.deep_box ? (s.D - t.t0) : a.deep_box;
+        int end;
+        if (lt < s.nds) {  // attention-sink tiles of a windowed draft
+            t.t0 = lt * a.deep_box;
+            end = s.se;
+        } else {
+            t.t0 = s.dw0 + (lt - s.nds) * a.deep_box;
+            end = s.D;
+        }
+        t.cnt = (end - t.t0) < a.deep_box ? (end - t.t0) : a.deep_box;
         t.y = t.t0;
         t.plane = a.R - 1;
         return t;
@@ -398,7 +418,7 @@ int max_active_clusters(void (*kern)(KArgs...), dim3 block, size_t smem, int clu
 int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, float *lse,
                   float scale, cudaStream_t s, const void *blk_k = nullptr, const void *blk_v = nullptr);
 int launch_draft(ripe_cache *c, int layer, int r, int j, const void *k, const void *v, const void *q, void *out,
-                 float *lse, float scale, cudaStream_t s);
+                 float *lse, float scale, cudaStream_t s, int sink = 0, int window = -1);
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q,
                        void *out, float *lse, float scale, cudaStream_t s);
 int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const void *v,

@@ -145,6 +145,9 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.plan.W = W;
     rv.plan.B = v->block_len;
     rv.plan.R = R;
+    rv.plan.sink = 0;
+    rv.plan.dwin = -1;
+    rv.plan.dj = 0;
     rv.plan.nloops = 1;
     rv.plan.loop[0] = static_cast<uint8_t>(r);
     for (int j = 0; j < kMaxQueryRows; ++j) rv.plan.jloop[j] = static_cast<uint8_t>(r);

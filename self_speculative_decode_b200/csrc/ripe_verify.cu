@@ -821,6 +821,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                                   (pa.mode_eff != 0 || tpos >= dsc.T || tpos >= pq - pa.W);
                         else if (dsc.kind == kDual)
                             vis = vis && tpos < pq - pa.W;
+                        if constexpr (FUSED) {  // windowed draft: sink and sliding window only
+                            if (pa.dwin >= 0) vis = vis && (tpos < pa.sink || tpos >= pq - pa.dwin);
+                        }
                         v = vis ? v : -INFINITY;
                     }
                     x[sb][nq][e] = v;
@@ -1110,7 +1113,8 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
 
 // One loop r; block positions [0, B) in the tile plan, queries at positions j0 .. j0 + qB - 1.
 static int launch_single_loop(ripe_cache *c, int layer, int r, int B, int j0, int qB, const void *q, void *out,
-                              float *lse, float scale, cudaStream_t s, const void *blk_k, const void *blk_v) {
+                              float *lse, float scale, cudaStream_t s, const void *blk_k, const void *blk_v,
+                              int sink = 0, int dwin = -1) {
     VerifyArgs a;
     a.blk_k = static_cast<const uint4 *>(blk_k);
     a.blk_v = static_cast<const uint4 *>(blk_v);
@@ -1122,6 +1126,9 @@ static int launch_single_loop(ripe_cache *c, int layer, int r, int B, int j0, in
     a.plan.W = c->W;
     a.plan.B = B;
     a.plan.R = c->R;
+    a.plan.sink = sink;
+    a.plan.dwin = dwin;
+    a.plan.dj = j0;
     a.plan.ring_slots = c->ring_slots;
     a.plan.deep_box = c->deep_box;
     a.plan.ring_box = c->ring_box;
@@ -1140,8 +1147,8 @@ int launch_verify(ripe_cache *c, int layer, int r, const void *q, void *out, flo
 
 // Draft step: position j of the block at loop r, its K/V written by the same launch.
 int launch_draft(ripe_cache *c, int layer, int r, int j, const void *k, const void *v, const void *q, void *out,
-                 float *lse, float scale, cudaStream_t s) {
-    return launch_single_loop(c, layer, r, j + 1, j, 1, q, out, lse, scale, s, k, v);
+                 float *lse, float scale, cudaStream_t s, int sink, int window) {
+    return launch_single_loop(c, layer, r, j + 1, j, 1, q, out, lse, scale, s, k, v, sink, window);
 }
 
 // Several loops in one call: block position j is verified at loop loop_of_position[j].
@@ -1157,6 +1164,9 @@ int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position
     a.plan.W = c->W;
     a.plan.B = c->B_cur;
     a.plan.R = c->R;
+    a.plan.sink = 0;
+    a.plan.dwin = -1;
+    a.plan.dj = 0;
     a.plan.ring_slots = c->ring_slots;
     a.plan.deep_box = c->deep_box;
     a.plan.ring_box = c->ring_box;

@@ -23,7 +23,7 @@ EXPORTS = (
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
     "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave", "ripe_append_verify",
-    "ripe_draft_attn",
+    "ripe_draft_attn", "ripe_draft_attn_window",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
             "ripe_append_verify": ([vp, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
             "ripe_draft_attn": ([vp, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
+            "ripe_draft_attn_window": ([vp, i, i, i, i, i, vp, vp, vp, vp, vp, ctypes.c_float, vp], i),
         }
         for name, (args, res) in sig.items():
             fn = getattr(L, name)
@@ -167,6 +168,12 @@ def ripe_draft_attn(h, layer, r, j, k, v, q, out, lse=None, scale=1.0, stream=No
     _check(lib().ripe_draft_attn(h, layer, r, j, ctypes.c_void_p(k), ctypes.c_void_p(v), ctypes.c_void_p(q),
                                  ctypes.c_void_p(out), ctypes.c_void_p(lse or 0), float(scale),
                                  _stream(stream)), "ripe_draft_attn")
+
+
+def ripe_draft_attn_window(h, layer, r, j, sink, window, k, v, q, out, lse=None, scale=1.0, stream=None):
+    _check(lib().ripe_draft_attn_window(h, layer, r, j, int(sink), int(window), ctypes.c_void_p(k), ctypes.c_void_p(v),
+                                        ctypes.c_void_p(q), ctypes.c_void_p(out), ctypes.c_void_p(lse or 0),
+                                        float(scale), _stream(stream)), "ripe_draft_attn_window")
 
 
 def ripe_verify_attn_wave(h, layer, loop_of_position, q, out, lse=None, scale=1.0, stream=None):
@@ -291,9 +298,11 @@ class RipeCache:
         ripe_append_verify(self.handle, layer, r, B, kp, vp, qp, op, lp, scale, stream)
         return out
 
-    def draft_attn(self, layer, r, j, k, v, q, out=None, lse=None, scale=1.0, stream=None):
+    def draft_attn(self, layer, r, j, k, v, q, out=None, lse=None, scale=1.0, stream=None, sink=None,
+                   window=None):
         """Draft step: write plane r of block position j (k, v [N][1][kvH][d]) and attend its
-        query q [N][1][Hq][d] over keys up to that position."""
+        query q [N][1][Hq][d] over keys up to that position; with ``sink`` / ``window`` only
+        over the first ``sink`` keys and the last ``window`` + 1 (windowed draft attention)."""
         import torch
         kshape = (self.N, 1, self.kvH, self.d)
         shape = (self.N, 1, self.Hq, self.d)
@@ -304,7 +313,11 @@ class RipeCache:
             out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
         op = _dev(out, torch.bfloat16, shape, "out").value
         lp = _dev(lse, torch.float32, shape[:3], "lse").value if lse is not None else None
-        ripe_draft_attn(self.handle, layer, r, j, kp, vp, qp, op, lp, scale, stream)
+        if sink is None and window is None:
+            ripe_draft_attn(self.handle, layer, r, j, kp, vp, qp, op, lp, scale, stream)
+        else:
+            ripe_draft_attn_window(self.handle, layer, r, j, 0 if sink is None else sink,
+                                   (1 << 30) if window is None else window, kp, vp, qp, op, lp, scale, stream)
         return out
 
     def verify_attn_wave(self, layer, loop_of_position, q, out=None, lse=None, scale=1.0, stream=None):

@@ -112,3 +112,36 @@ def test_draft_redraft_and_state_errors(cuda_device):
     assert c.gpu.sync_lengths() == [92, 34]
     step(0)                      # a new draft phase after the commit
     c.close()
+
+
+@pytest.mark.parametrize("kw,sink,window", [
+    (dict(N=2, Hq=4, kvH=2, d=128, R=4, T=[700, 300], W=16, B=6), 4, 40),      # window reaches the deep region
+    (dict(N=2, Hq=3, kvH=3, d=96, R=3, T=[900, 77], W=32, B=8), 100, 10),      # two sink tiles; sink covers seq 1
+    (dict(N=1, Hq=2, kvH=2, d=64, R=3, T=[500], W=0, B=4), 1, 0),              # deepest only: sink + the query
+    (dict(N=2, Hq=60, kvH=30, d=96, R=4, T=[600, 600], W=16, B=8), 4, 200),    # two CTAs per head
+    (dict(N=1, Hq=2, kvH=2, d=64, R=3, T=[300], W=10 ** 6, B=5), 8, 64),       # full cache
+])
+def test_windowed_draft_parity(kw, sink, window, cuda_device):
+    """Windowed draft attention (attention sink + sliding window on the draft only) against the
+    oracle; with a window reaching position 0 it equals the plain draft step."""
+    c = Case(L=1, seed=43, independent=True, append_block=False, **kw)
+    idx_n = torch.tensor(c.oseq, device=c.device)
+    idx_h = torch.tensor(c.oheads, device=c.device)
+    loops = [0, kw["R"] - 1]
+    for j in range(kw["B"]):
+        for r in loops:
+            kb, vb = c.blocks[(0, r)]
+            k1, v1 = _rows(kb, j), _rows(vb, j)
+            q1 = _rows(c.src[0].queries(r, c.B, c.Hq, 0), j)
+            lse = torch.empty((c.N, 1, c.Hq), dtype=torch.float32, device=c.device)
+            out = c.gpu.draft_attn(0, r, j, c._dev(k1), c._dev(v1), c._dev(q1), lse=lse, sink=sink, window=window)
+            ro, rl = c.orc.draft(0, r, j, c._sub_block(k1), c._sub_block(v1),
+                                 np.ascontiguousarray(c._host(q1)[c.oseq][:, :, c.oheads]), c.g,
+                                 sink=sink, window=window)
+            check_close(out.index_select(0, idx_n).index_select(2, idx_h), ro, f"windowed draft j={j} loop {r}")
+            check_lse(lse.index_select(0, idx_n).index_select(2, idx_h), rl)
+            if j == 0:
+                full = c.gpu.draft_attn(0, r, j, c._dev(k1), c._dev(v1), c._dev(q1), sink=0, window=1 << 20)
+                plain = c.gpu.draft_attn(0, r, j, c._dev(k1), c._dev(v1), c._dev(q1))
+                assert torch.equal(full, plain)
+    c.close()

@@ -366,3 +366,55 @@ def test_draft_state_rules():
     assert int(c.T[0]) == T + 1
     assert not c.present[0, :, 0, T + 1:].any()    # rejected block rows and drafts past the block
     assert c.drafted.sum() == 0
+
+
+# ---------------------------------------------------------------- windowed draft attention
+def test_windowed_draft_without_restriction_is_the_draft():
+    """sink = 0 and a window reaching position 0: every key is attended, as in the draft."""
+    N, kvH, g, d, R, W, T, B = 2, 2, 2, 8, 4, 5, 30, 4
+    c, PK, PV, src = _prefix_cache(N, kvH, g, d, R, W, T, B, seed=29)
+    kb, vb = block_from_planes(PK[1], T, B), block_from_planes(PV[1], T, B)
+    q = src.queries(1, B, kvH * g)
+    for j in range(B):
+        a, la = c.draft(0, 1, j, kb[:, j:j + 1], vb[:, j:j + 1], q[:, j:j + 1], g, 1.1)
+        b, lb = c.draft(0, 1, j, kb[:, j:j + 1], vb[:, j:j + 1], q[:, j:j + 1], g, 1.1, sink=0, window=T + j)
+        assert np.abs(a - b).max() < 1e-12 and np.abs(la - lb).max() < 1e-12
+
+
+@pytest.mark.parametrize("window", [0, 1, 3, 5])
+def test_windowed_draft_inside_the_ripe_window_is_sdpa_on_plane_r(window):
+    """No sink and a draft window no longer than the RIPE window: every attended key reads plane
+    r, so the result is textbook attention over keys [p - window, p] of plane r (torch SDPA)."""
+    N, kvH, g, d, R, W, T, B = 1, 2, 2, 8, 4, 5, 30, 3
+    r = 1
+    c, PK, PV, src = _prefix_cache(N, kvH, g, d, R, W, T, B, seed=31)
+    kb, vb = block_from_planes(PK[r], T, B), block_from_planes(PV[r], T, B)
+    q = src.queries(r, B, kvH * g)
+    for j in range(B):
+        out, _ = c.draft(0, r, j, kb[:, j:j + 1], vb[:, j:j + 1], q[:, j:j + 1], g, 1.0, sink=0, window=window)
+        p = T + j
+        K = _f64(PK[r][0, :, p - window:p + 1])          # [kvH][window+1][d], plane r
+        V = _f64(PV[r][0, :, p - window:p + 1])
+        qt = torch.from_numpy(_f64(q[0, j]))[:, None, :]  # [Hq][1][d]
+        kt = torch.from_numpy(K).repeat_interleave(g, dim=0)
+        vt = torch.from_numpy(V).repeat_interleave(g, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=1.0)[:, 0].numpy()
+        assert np.abs(out[0, 0] - ref).max() < 1e-12
+
+
+def test_windowed_draft_ignores_keys_between_sink_and_window():
+    """Keys between the sink and the window do not enter the result; sink and window keys do."""
+    N, kvH, g, d, R, W, T, B = 1, 1, 1, 8, 3, 4, 40, 2
+    c, PK, PV, src = _prefix_cache(N, kvH, g, d, R, W, T, B, seed=37)
+    kb, vb = block_from_planes(PK[0], T, B), block_from_planes(PV[0], T, B)
+    q = src.queries(0, B, 1)
+    sink, window = 3, 6
+    base, _ = c.draft(0, 0, 0, kb[:, :1], vb[:, :1], q[:, :1], g, 1.0, sink=sink, window=window)
+    for t, inside in ((10, False), (25, False), (1, True), (T - 2, True)):
+        plane = R - 1 if t < T - W else 0
+        saved = c.values(0, plane, "V")[0, 0, t].copy()
+        bumped = (_f64(saved) + 3.0).astype(np.float32).view(np.uint32) >> np.uint32(16)
+        c.values(0, plane, "V")[0, 0, t] = bumped.astype(np.uint16)   # that value + 3
+        moved, _ = c.draft(0, 0, 0, kb[:, :1], vb[:, :1], q[:, :1], g, 1.0, sink=sink, window=window)
+        c.values(0, plane, "V")[0, 0, t] = saved
+        assert (np.abs(moved - base).max() > 1e-6) == inside, t
