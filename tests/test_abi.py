@@ -58,5 +58,10 @@ def test_calls_on_a_null_handle_are_rejected():
     assert L.ripe_verify_attn(null, 0, 0, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
     assert L.ripe_append_block(null, 0, 0, 1, null, null, null) == ripe.RIPE_EINVAL
     assert L.ripe_commit(null, None, null) == ripe.RIPE_EINVAL
+    assert L.ripe_append_verify(null, 0, 0, 1, null, null, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
+    assert L.ripe_draft_attn(null, 0, 0, 0, null, null, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
+    assert L.ripe_draft_attn_window(null, 0, 0, 0, 4, 64, null, null, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
+    assert L.ripe_draft_attn_window(null, 0, 0, 0, -1, 64, null, null, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
+    assert L.ripe_verify_attn_wave(null, 0, None, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
     assert L.ripe_cache_free(null) == ripe.RIPE_OK
     assert L.ripe_launch_count(null) == -1
