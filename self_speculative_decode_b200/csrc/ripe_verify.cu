@@ -377,7 +377,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const uint32_t empty0 = smem_addr(&bars[NS]);
     const uint32_t stage0 = smem_addr(stages);
 
-    // FUSED (ripe_append_verify): the consumers first write the draft block into the ring; a
+    // FUSED (ripe_append_verify, draft steps): a copy warp writes the block rows into the ring; a
     // separate instantiation so that plain verification carries none of that code
     constexpr bool fused = FUSED;
     if constexpr (fused) {
@@ -412,7 +412,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             int i = 0;
             bool ok = true;
             // with a fused append, the tiles holding the rows this launch writes wait until the
-            // consumers have written them: the loop below runs in two phases, up to the first such
+            // copy warp has written them: the loop below runs in two phases, up to the first such
             // tile of the chunk and from it, and stays free of a per-tile check
             int bound = ntiles;
             if (fused) bound = first_written_tile(sg, lt, n, kh, ntiles, Ts, a);
@@ -463,7 +463,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 }
             }
             if (!ok || bound >= ntiles) break;
-            // the consumers wrote the block's rows into the ring (generic proxy) and fenced them
+            // the copy warp wrote the block's rows into the ring (generic proxy) and fenced them
             if (!mbar_wait_bounded(smem_addr(&bars[2 * NS]), 0)) {
                 ok = false;
                 break;
