@@ -308,7 +308,8 @@ def _prefix_cache(N, kvH, g, d, R, W, T, B, seed, max_extra=0):
     return c, PK, PV, src
 
 
-@pytest.mark.parametrize("T,W,B,r,g", [(20, 3, 5, 0, 2), (20, 0, 4, 1, 1), (6, 10, 4, 2, 3), (15, 5, 6, 4, 1)])
+@pytest.mark.parametrize("T,W,B,r,g", [(20, 3, 5, 0, 2), (20, 0, 4, 1, 1), (6, 10, 4, 2, 3), (15, 5, 6, 4, 1),
+                                       (0, 3, 4, 0, 1), (1, 0, 3, 2, 2)])
 def test_draft_steps_match_the_brute_force(T, W, B, r, g):
     """Draft step j (one query at p = T + j, the drafts 0..j at plane r) equals row j of the
     independent brute-force formulation over the same planes; the drafted rows then verified
