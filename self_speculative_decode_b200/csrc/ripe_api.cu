@@ -140,7 +140,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     c->kv_bytes = c->scratch_bytes = 0;
     c->launches = 0;
 
-    if (cudaGetDevice(&c->device) != cudaSuccess ||
+    if (cudaGetDevice(&c->device) != cudaSuccess || c->device >= kMaxDevices ||
         cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
         cudaGetLastError();
         delete c;
@@ -176,7 +176,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     }
     ok = ok && encode_map(&c->tm_Kw, c->Kw, head_dim, c->ring_slots, ring_pages, c->ring_box) &&
          encode_map(&c->tm_Vw, c->Vw, head_dim, c->ring_slots, ring_pages, c->ring_box);
-    if (!ok || set_verify_attributes(head_dim, batch) != RIPE_OK || cudaDeviceSynchronize() != cudaSuccess) {
+    if (!ok || ensure_verify_attributes(c->device) != RIPE_OK || cudaDeviceSynchronize() != cudaSuccess) {
         cudaGetLastError();
         release(c);
         return RIPE_ECUDA;

@@ -19,6 +19,7 @@ constexpr int kBoxCols = 32;      // bf16 per TMA box row: 64 bytes, 64-byte swi
 constexpr int kBoxBytes = kTileRows * 64;  // one box slot in shared memory (4 KB)
 constexpr int kStages = 4;        // TMA pipeline depth of the verify kernel
 constexpr int kMaxQueryRows = 64; // B * (Hq / kvH) per key/value head
+constexpr int kMaxDevices = 64;   // devices a process may drive (per-device set-up tables)
 
 // Bounded waits: a kernel that does not see its copies land within this time records
 // RIPE_DEVERR_WAIT_TIMEOUT and stops (it never traps).
@@ -428,7 +429,9 @@ int launch_load_prefix(ripe_cache *c, int layer, int plane, const int32_t *T, co
                        const void *v, int64_t ld_t, cudaStream_t s);
 int launch_export(ripe_cache *c, int n, int layer, void *k_out, void *v_out, uint8_t *present,
                   cudaStream_t s);
-int set_verify_attributes(int d, int N);
+// Raise the verify kernels' dynamic shared-memory limit on `device` (which must be current) to
+// what the largest batch needs; once per device, thread-safe.
+int ensure_verify_attributes(int device);
 
 // Everything one verify launch needs, for callers that own the buffers and the scratch.
 struct RawVerify {
@@ -442,6 +445,7 @@ struct RawVerify {
     uint32_t *err;
     PlanArgs plan;
     int N, kvH, g, Hq, d, layer, grid, has_deep;
+    int device, num_sms;
     float scale;
 };
 int launch_verify_raw(const RawVerify &rv, cudaStream_t s);

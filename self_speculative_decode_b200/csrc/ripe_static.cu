@@ -13,7 +13,7 @@
 
 namespace {
 
-constexpr int kMaxDevices = 64;
+using ripe::kMaxDevices;
 
 __device__ __align__(256) unsigned char g_static_scratch[RIPE_STATIC_SCRATCH_BYTES];
 
@@ -25,7 +25,8 @@ struct DeviceSetup {
 DeviceSetup g_setup[kMaxDevices];
 std::mutex g_setup_mu;
 
-// Once per device, with that device current: the array's device address and the SM count.
+// Once per device, with that device current: the array's device address, the SM count, and the
+// verify kernels' shared-memory limit.
 // (In host code the array's name is only a host-side stand-in, never a device address.)
 int setup_device(int dev, DeviceSetup *&out) {
     if (dev < 0 || dev >= kMaxDevices) return RIPE_EINVAL;
@@ -42,6 +43,9 @@ int setup_device(int dev, DeviceSetup *&out) {
             cudaGetLastError();
             return RIPE_ECUDA;
         }
+        // the kernels' shared-memory limit (shared with caches on this device; only ever raised)
+        const int st = ripe::ensure_verify_attributes(dev);
+        if (st != RIPE_OK) return st;
         s.scratch = static_cast<unsigned char *>(p);
         s.num_sms = sms;
         s.done = true;
@@ -162,6 +166,8 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.d = d;
     rv.layer = layer;
     rv.grid = grid;
+    rv.device = dev;
+    rv.num_sms = ds->num_sms;
     rv.has_deep = deep_rows > 0 ? 1 : 0;
     rv.scale = scale;
     const int ls = launch_verify_raw(rv, s);

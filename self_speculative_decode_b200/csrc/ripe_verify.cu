@@ -32,6 +32,7 @@
 //     scratch; the last to arrive (atomic counter, no spinning) merges them.
 //   * Every wait is bounded: on timeout the kernel records RIPE_DEVERR_WAIT_TIMEOUT, drains
 //     its own copies in flight and returns without writing further results.
+#include <mutex>
 #include <type_traits>
 
 #include "ripe_common.cuh"
@@ -938,57 +939,72 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 }
 
 // ---------------------------------------------------------------- host side
+// The per-function limit on dynamic shared memory.  A launch asks for smem_bytes_for<C>(N),
+// which grows with the batch N (the per-sequence tile counts live in shared memory).  The
+// limit is raised once per device to what the largest batch asks for, so that no cache
+// allocation or call ever lowers it below what a live cache of a larger batch needs.
+template <class C>
+constexpr int kSmemMax = smem_bytes_for<C>(kMaxBatch);
+
+// Where a verify launch reads from: the four tensor maps, the device and its SM count.
+struct LaunchTarget {
+    const CUtensorMap *tmKd, *tmVd, *tmKw, *tmVw;
+    int device, num_sms, N;
+};
+
 template <int D, int NQT, int WR, int WK, int TG>
 struct Inst {
     using C = VCfg<D, NQT, WR, WK, TG>;
+    static_assert(kSmemMax<C> <= kSmemLimit, "the largest batch's shared memory must fit a CTA");
     static constexpr auto kernel = ripe_verify_kernel<D, NQT, WR, WK, TG, false>;
     static constexpr auto kernel_fused = ripe_verify_kernel<D, NQT, WR, WK, TG, true>;
-    static cudaError_t set_attr(int N) {
-        const int bytes = smem_bytes_for<C>(N);
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    static cudaError_t set_attr_max() {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax<C>);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(kernel_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            e = cudaFuncSetAttribute(kernel_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax<C>);
         return e;
     }
-    // 2 x the clusters of two CTAs that fit at once (0: no cluster launch), per instance and
-    // shared-memory size
-    static int pair_grid(bool fused, int smem, int num_sms) {
-        static int cached_smem[2] = {-1, -1}, cached[2] = {0, 0};
+    // 2 x the clusters of two CTAs that fit at once (0: no cluster launch), per device, instance
+    // and shared-memory size
+    static int pair_grid(bool fused, int smem, int device, int num_sms) {
+        struct Entry {
+            int smem = -1, grid = 0;
+        };
+        static Entry cache[kMaxDevices][2];
+        static std::mutex mu;
         const int f = fused ? 1 : 0;
-        if (cached_smem[f] != smem) {
+        std::lock_guard<std::mutex> lock(mu);
+        Entry &e = cache[device][f];
+        if (e.smem != smem) {
             const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::THREADS + 32 * f), smem, 2,
                                               num_sms & ~1);
-            cached[f] = 2 * n;
-            cached_smem[f] = smem;
+            e.grid = 2 * n;
+            e.smem = smem;
         }
-        return cached[f];
+        return e.grid;
     }
-    static void launch(const ripe_cache *c, int grid, const VerifyArgs &args, cudaStream_t s) {
+    static cudaError_t launch(const LaunchTarget &t, int grid, const VerifyArgs &args, cudaStream_t s) {
         if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
         const bool fused = args.blk_k != nullptr;
         auto kern = fused ? kernel_fused : kernel;
         const dim3 block(C::THREADS + (fused ? 32 : 0));
-        const int smem = smem_bytes_for<C>(c->N);
+        const int smem = smem_bytes_for<C>(t.N);
         VerifyArgs a = args;
         a.xpair = 0;
 #ifndef RIPE_NO_XPAIR
         if (C::XPAIR) {
-            const int pg = pair_grid(fused, smem, c->num_sms);
+            const int pg = pair_grid(fused, smem, t.device, t.num_sms);
             if (pg >= 2) {
                 int g2 = (grid + 1) & ~1;
                 if (g2 > pg) g2 = pg;
                 a.xpair = 1;
-                launch_pdl_cluster(kern, dim3(g2), block, smem, s, 2, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
-                return;
+                return launch_pdl_cluster(kern, dim3(g2), block, smem, s, 2, *t.tmKd, *t.tmVd, *t.tmKw, *t.tmVw, a);
             }
         }
 #endif
-        launch_pdl(kern, dim3(grid), block, smem, s, c->tm_Kd, c->tm_Vd, c->tm_Kw, c->tm_Vw, a);
+        return launch_pdl(kern, dim3(grid), block, smem, s, *t.tmKd, *t.tmVd, *t.tmKw, *t.tmVw, a);
     }
 };
-
-template <class I>
-constexpr auto ripe_verify_kernel_of() { return I::kernel; }
 
 // query-side configuration by the number of query rows per kv head (B * group)
 //   <= 8  : one 8-query tile per warp, 2 tile groups of 4 warps
@@ -1013,63 +1029,53 @@ constexpr auto ripe_verify_kernel_of() { return I::kernel; }
 static int qcfg_of(int Mq) { return Mq <= 8 ? 0 : Mq <= 16 ? 1 : Mq <= 32 ? 2 : 3; }
 
 template <class... I>
-static cudaError_t set_all(int N) {
+static cudaError_t set_all_max() {
     cudaError_t e = cudaSuccess;
-    ((e = (e == cudaSuccess ? I::set_attr(N) : e)), ...);
+    ((e = (e == cudaSuccess ? I::set_attr_max() : e)), ...);
     return e;
 }
 
-int set_verify_attributes(int d, int N) {
-    cudaError_t e;
+int ensure_verify_attributes(int device) {
+    if (device < 0 || device >= kMaxDevices) return RIPE_EINVAL;
+    static bool done[kMaxDevices] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[device]) return RIPE_OK;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != device) return RIPE_ECUDA;  // caller makes it current
+    cudaError_t e = set_all_max<RIPE_QCFG_LIST(64)>();
+    if (e == cudaSuccess) e = set_all_max<RIPE_QCFG_LIST(96)>();
+    if (e == cudaSuccess) e = set_all_max<RIPE_QCFG_LIST(128)>();
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return RIPE_ECUDA;
+    }
+    done[device] = true;
+    return RIPE_OK;
+}
+
+template <class I0, class I1, class I2, class I3>
+static cudaError_t launch_d(int qc, const LaunchTarget &t, int grid, const VerifyArgs &a, cudaStream_t s) {
+    switch (qc) {
+        case 0: return I0::launch(t, grid, a, s);
+        case 1: return I1::launch(t, grid, a, s);
+        case 2: return I2::launch(t, grid, a, s);
+        default: return I3::launch(t, grid, a, s);
+    }
+}
+
+static cudaError_t launch_any(int d, int qc, const LaunchTarget &t, int grid, const VerifyArgs &a, cudaStream_t s) {
     switch (d) {
-        case 64: e = set_all<RIPE_QCFG_LIST(64)>(N); break;
-        case 96: e = set_all<RIPE_QCFG_LIST(96)>(N); break;
-        case 128: e = set_all<RIPE_QCFG_LIST(128)>(N); break;
-        default: return RIPE_EINVAL;
-    }
-    return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
-}
-
-template <class I0, class I1, class I2, class I3>
-static void launch_d(int qc, const ripe_cache *c, int grid, const VerifyArgs &a, cudaStream_t s) {
-    switch (qc) {
-        case 0: I0::launch(c, grid, a, s); break;
-        case 1: I1::launch(c, grid, a, s); break;
-        case 2: I2::launch(c, grid, a, s); break;
-        default: I3::launch(c, grid, a, s); break;
-    }
-}
-
-// Launch over explicitly given buffers and scratch (the allocation-free entry point).
-template <class I0, class I1, class I2, class I3>
-static cudaError_t launch_raw_d(int qc, const RawVerify &rv, const VerifyArgs &a, cudaStream_t s) {
-    switch (qc) {
-        case 0: return launch_pdl(ripe_verify_kernel_of<I0>(), dim3(rv.grid < I0::C::MAX_PARTS ? rv.grid : I0::C::MAX_PARTS), dim3(I0::C::THREADS),
-                                  smem_bytes_for<typename I0::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        case 1: return launch_pdl(ripe_verify_kernel_of<I1>(), dim3(rv.grid < I1::C::MAX_PARTS ? rv.grid : I1::C::MAX_PARTS), dim3(I1::C::THREADS),
-                                  smem_bytes_for<typename I1::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        case 2: return launch_pdl(ripe_verify_kernel_of<I2>(), dim3(rv.grid < I2::C::MAX_PARTS ? rv.grid : I2::C::MAX_PARTS), dim3(I2::C::THREADS),
-                                  smem_bytes_for<typename I2::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-        default: return launch_pdl(ripe_verify_kernel_of<I3>(), dim3(rv.grid < I3::C::MAX_PARTS ? rv.grid : I3::C::MAX_PARTS), dim3(I3::C::THREADS),
-                                   smem_bytes_for<typename I3::C>(rv.N), s, rv.tmKd, rv.tmVd, rv.tmKw, rv.tmVw, a);
-    }
-}
-
-template <class I>
-static cudaError_t set_attr_raw(int N) { return I::set_attr(N); }
-
-template <class I0, class I1, class I2, class I3>
-static cudaError_t set_raw_d(int qc, int N) {
-    switch (qc) {
-        case 0: return set_attr_raw<I0>(N);
-        case 1: return set_attr_raw<I1>(N);
-        case 2: return set_attr_raw<I2>(N);
-        default: return set_attr_raw<I3>(N);
+        case 64: return launch_d<RIPE_QCFG_LIST(64)>(qc, t, grid, a, s);
+        case 96: return launch_d<RIPE_QCFG_LIST(96)>(qc, t, grid, a, s);
+        case 128: return launch_d<RIPE_QCFG_LIST(128)>(qc, t, grid, a, s);
+        default: return cudaErrorInvalidValue;
     }
 }
 
 int verify_rows_for(int Mq) { return 8 << qcfg_of(Mq); }
 
+// Launch over explicitly given buffers and scratch (the allocation-free entry point).
 int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     VerifyArgs a;
     a.blk_k = a.blk_v = nullptr;
@@ -1098,17 +1104,10 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.min_chunk = RIPE_MIN_CHUNK;
     a.has_deep = rv.has_deep;
     a.scale_log2 = rv.scale * 1.4426950408889634f;
-    const int qc = qcfg_of(a.Mq);
-    cudaError_t e;
-    switch (rv.d) {
-        case 64: e = set_raw_d<RIPE_QCFG_LIST(64)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(64)>(qc, rv, a, s); break;
-        case 96: e = set_raw_d<RIPE_QCFG_LIST(96)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(96)>(qc, rv, a, s); break;
-        case 128: e = set_raw_d<RIPE_QCFG_LIST(128)>(qc, rv.N); if (!e) e = launch_raw_d<RIPE_QCFG_LIST(128)>(qc, rv, a, s); break;
-        default: return RIPE_EINVAL;
-    }
-    return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
+    const LaunchTarget t = {&rv.tmKd, &rv.tmVd, &rv.tmKw, &rv.tmVw, rv.device, rv.num_sms, rv.N};
+    if (rv.d != 64 && rv.d != 96 && rv.d != 128) return RIPE_EINVAL;
+    return launch_any(rv.d, qcfg_of(a.Mq), t, rv.grid, a, s) == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
-
 static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s);
 
 // One loop r; block positions [0, B) in the tile plan, queries at positions j0 .. j0 + qB - 1.
@@ -1212,14 +1211,11 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
         if (need < grid) grid = static_cast<int>(need);
     }
     if (grid < 1) grid = 1;
-    switch (c->d) {
-        case 64: launch_d<RIPE_QCFG_LIST(64)>(qc, c, grid, a, s); break;
-        case 96: launch_d<RIPE_QCFG_LIST(96)>(qc, c, grid, a, s); break;
-        case 128: launch_d<RIPE_QCFG_LIST(128)>(qc, c, grid, a, s); break;
-        default: return RIPE_EINVAL;
-    }
+    if (c->d != 64 && c->d != 96 && c->d != 128) return RIPE_EINVAL;
+    const LaunchTarget t = {&c->tm_Kd, &c->tm_Vd, &c->tm_Kw, &c->tm_Vw, c->device, c->num_sms, c->N};
+    const cudaError_t e = launch_any(c->d, qc, t, grid, a, s);
     c->launches += 1;
-    return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
+    return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 
 }  // namespace ripe

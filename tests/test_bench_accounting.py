@@ -40,3 +40,37 @@ def test_windowed_draft_bytes_cover_the_attended_keys(T, W, j, sink, window):
     attended = [t for t in range(p + 1) if t < sink or t >= p - window]
     read_rows = (bench.draft_window_bytes(cfg, [T], r, j, W, sink, window) - 4) // 4
     assert len(attended) <= read_rows <= len(attended) + W + j + bench.dual_keys(T, W, j + 1, R, r)
+
+
+def test_fixed_memory_batch_fit():
+    """The largest batch whose key/value regions fit a budget: floor(budget / bytes per sequence),
+    capped at the library's batch limit."""
+    assert bench.fit_batch(3.18e9, 20e9) == 6
+    assert bench.fit_batch(289e6, 20e9) == 69
+    assert bench.fit_batch(121e6, 20e9) == 165
+    assert bench.fit_batch(10, 1e9) == 1024                    # capped
+    assert bench.fit_batch(21e9, 20e9) == 0                    # one sequence does not fit
+    with pytest.raises(ValueError):
+        bench.fit_batch(0, 1e9)
+
+
+def test_two_point_cost_model_recovers_a_line():
+    """t(N) = a + b N through two measured points gives back a and b exactly for a linear cost, and
+    predicts the third point."""
+    a, b = 0.8, 0.57
+    t = lambda n: a + b * n
+    fa, fb = bench.two_point_cost_model(t(1), t(138), 138)
+    assert abs(fa - a) < 1e-12 and abs(fb - b) < 1e-12
+    assert abs(fa + fb * 40 - t(40)) < 1e-12
+    assert bench.two_point_cost_model(2.0, 2.0, 1) == (2.0, 0.0)
+
+
+def test_l2_note_classifies_working_sets():
+    l2 = 126 * 2 ** 20
+    assert "both stream from HBM" in bench.l2_note(1.07e9, 4.5e9, l2)        # long-context call
+    assert "partly served" in bench.l2_note(22e6, 300e6, l2)                  # Huginn call, step > L2
+    assert "largely from L2" in bench.l2_note(1e6, 50e6, l2)                  # tiny
+    # the step's distinct bytes: deepest region once per layer plus every loop's window ring
+    cfg = dict(N=1, kvH=55, d=96, R=32, B=8)
+    row = 4 * 55 * 96
+    assert bench.step_distinct_bytes(cfg, 1024, 64, 4) == 4 * row * (960 + 32 * 72)

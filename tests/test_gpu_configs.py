@@ -5,9 +5,10 @@
   against the oracle, and block-split independence checked on the GPU for every W >= B-1;
 * long-context GQA: 32 q / 8 kv heads x 128, R=32, T=32768, W=64, B=8, batch 8, rho 0.85
   (one layer of four), RIPE and full-cache layouts;
-* streaming decode: 16 sequences, Huginn heads, R=32, W=64, B=8, T0=512, accepted lengths
-  drawn U{0..8} per step, fresh drafts every step: verify parity on sampled steps, loops,
-  sequences and heads, and the exported cache state bit-exact against the oracle's;
+* streaming decode: 16 sequences, Huginn heads, R=32, W=64, B=8, accepted lengths drawn
+  U{0..8} per step, fresh drafts every step, from T0=512 and from ragged lengths near 4000
+  (where 1000 steps end): verify parity on sampled steps, loops, sequences and heads, and the
+  exported cache state bit-exact against the oracle's;
 * edge shapes: B=1 (draft-phase decode), R=1, 64 query rows per kv head.
 """
 import numpy as np
@@ -108,25 +109,30 @@ def test_long_context_gqa_sampled(layout, cuda_device):
     c.close()
 
 
-def test_streaming_decode_with_maintenance(cuda_device):
-    N, kvH, d, R, W, B, T0, steps = 16, 55, 96, 32, 64, 8, 512, 24
+def _streaming(T0, steps, seed, device):
+    """16 sequences, Huginn heads, R=32, W=64, B=8 from committed lengths T0 (one per sequence):
+    fresh block planes every step, accepted lengths U{0..8}; verify parity on sampled steps, loops,
+    sequences and heads, then the exported cache state bit for bit."""
+    N, kvH, d, R, W, B = 16, 55, 96, 32, 64, 8
     loops_checked = [0, 31]
     seqs, heads = [0, 5, 15], [0, 54]
-    acc = acceptance_draws(3, steps, N, B)
-    max_T = T0 + B * (steps + 1)
-    src = PlaneSource(N, kvH, d, R, T0, 0.88, 3, backend="torch", device=cuda_device)
+    acc = acceptance_draws(seed, steps, N, B)
+    max_T = max(T0) + B * (steps + 1)
+    src = PlaneSource(N, kvH, d, R, max(T0), 0.88, seed, backend="torch", device=device)
     gpu = RipeCache(N, 1, kvH, kvH, d, R, W, max_T, B)
     oc = orc.OracleCache(len(seqs), 1, len(heads), d, R, W, max_T, value_planes=set(loops_checked))
     sub = lambda x: np.ascontiguousarray(dev_to_bits(x)[seqs][:, heads])
     subb = lambda x: np.ascontiguousarray(dev_to_bits(x)[seqs][:, :, heads])
+    To = [T0[n] for n in seqs]
     for pl in range(R):
         k, v = src.plane(pl, "K"), src.plane(pl, "V")
-        gpu.load_prefix(0, pl, [T0] * N, k, v)
+        gpu.load_prefix(0, pl, T0, k, v)
         keep = pl in loops_checked
-        oc.load_prefix(0, pl, [T0] * len(seqs), sub(k) if keep else None, sub(v) if keep else None)
+        oc.load_prefix(0, pl, To, sub(k) if keep else None, sub(v) if keep else None)
+        del k, v
     src.release()
-    hsel = torch.tensor(heads, device=cuda_device)
-    nsel = torch.tensor(seqs, device=cuda_device)
+    hsel = torch.tensor(heads, device=device)
+    nsel = torch.tensor(seqs, device=device)
     for step in range(steps):
         for pl in range(R):
             kb, vb = src.block(step, pl, B, "K"), src.block(step, pl, B, "V")
@@ -137,28 +143,42 @@ def test_streaming_decode_with_maintenance(cuda_device):
                 oc.append(0, pl, None, None, B=B)
         for r in range(R):
             q = src.queries(r, B, kvH, step)
-            lse = torch.empty((N, B, kvH), dtype=torch.float32, device=cuda_device)
+            lse = torch.empty((N, B, kvH), dtype=torch.float32, device=device)
             out = gpu.verify_attn(0, r, q, lse=lse)
-            if r in loops_checked and step in (0, 11, steps - 1):
+            if r in loops_checked and step in (0, steps // 2, steps - 1):
                 ro, rl = oc.verify(0, r, subb(q), 1)
                 check_close(out.index_select(0, nsel).index_select(2, hsel), ro, f"step {step} loop {r}")
                 check_lse(lse.index_select(0, nsel).index_select(2, hsel), rl)
         gpu.commit(acc[step])
         oc.commit(acc[step][seqs])
     T = gpu.sync_lengths()
-    assert T == [T0 + int(x) for x in acc.sum(0)]
+    assert T == [T0[n] + int(x) for n, x in enumerate(acc.sum(0))]
     assert len(set(T)) > 1                       # ragged lengths
     for i, n in enumerate(seqs):                 # exported state of the sampled sequences, bit for bit
         k, v, present = gpu.export(n, 0)
         pres = oc.present[0, :, i, : T[n]]
         np.testing.assert_array_equal(present.cpu().numpy().astype(bool), pres)
-        kb = dev_to_bits(k)
+        kb, vbits = dev_to_bits(k), dev_to_bits(v)
         for pl in loops_checked:
-            ok = oc.values(0, pl, "K")[i, :, : T[n]]
             m = pres[pl][None, :, None]
-            np.testing.assert_array_equal(np.where(m, kb[pl][heads], 0), np.where(m, ok, 0))
+            for which, bits in (("K", kb), ("V", vbits)):
+                ok = oc.values(0, pl, which)[i, :, : T[n]]
+                np.testing.assert_array_equal(np.where(m, bits[pl][heads], 0), np.where(m, ok, 0))
     assert gpu.device_error() == 0
     gpu.close()
+
+
+def test_streaming_decode_with_maintenance(cuda_device):
+    """The streaming workload from its start: every sequence at T0 = 512."""
+    _streaming([512] * 16, 24, 3, cuda_device)
+
+
+def test_streaming_decode_late_lengths(cuda_device):
+    """The streaming workload near where it ends (about 4000 committed positions after 1000 steps
+    of U{0..8} accepted lengths): ragged starting lengths 3900..4400, 24 more steps."""
+    rng = np.random.default_rng(17)
+    T0 = [int(x) for x in rng.integers(3900, 4401, size=16)]
+    _streaming(T0, 24, 17, cuda_device)
 
 
 @pytest.mark.parametrize("kw", [

@@ -1,11 +1,12 @@
 """ripe_append_verify == ripe_append_block + ripe_verify_attn, bit for bit: the outputs of every
 call and the cache state after each commit, over several decode steps with ragged accepted
-lengths (ring wrap-around, eviction, all three layouts)."""
+lengths (ring wrap-around, eviction, all three layouts); and ripe_append_verify against the CPU
+oracle directly."""
 import numpy as np
 import pytest
 import torch
 
-from harness import dev_to_bits
+from harness import Case, check_close, check_lse, dev_to_bits
 from self_speculative_decode_b200.ripe import RipeCache
 from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
 
@@ -50,3 +51,21 @@ def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, T0, cuda_devic
     for c in caches:
         assert c.device_error() == 0
         c.close()
+
+
+@pytest.mark.parametrize("W", [16, 0, 10 ** 6])
+def test_fused_append_verify_against_the_oracle(W, cuda_device):
+    """Each plane of the block written by the verify launch itself, then checked against the
+    oracle (tagged planes: a wrong plane or a row written to the wrong slot is an O(1) error)."""
+    c = Case(N=3, L=1, Hq=6, kvH=3, d=96, R=4, T=[90, 7, 45], W=W, B=8, seed=33, independent=True,
+             append_block=False)
+    for r in range(4):
+        kb, vb = c.blocks[(0, r)]
+        qd, qh = c.queries(0, r)
+        lse = torch.empty((c.N, c.B, c.Hq), dtype=torch.float32, device=c.device)
+        out = c.gpu.append_verify(0, r, c._dev(kb), c._dev(vb), qd, lse=lse)
+        c.orc.append(0, r, c._sub_block(kb), c._sub_block(vb))
+        ro, rl = c.orc.verify(0, r, qh, c.g)
+        check_close(out, ro, f"fused loop {r}")
+        check_lse(lse, rl)
+    c.close()

@@ -140,6 +140,41 @@ def test_softmax_weights_sum_to_one():
     assert np.abs(out - 1.0).max() < 1e-12
 
 
+def test_softmax_weights_match_independent_formulations():
+    """oracle.weights against two formulations that share none of its code.
+
+    (1) brute_verify with one-hot values (the value of key t is e_t on every plane, d >= T + B):
+    its output row for query j is exactly that query's weight vector, computed from brute_verify's
+    own full-depth key sets and its own softmax.  (2) torch.softmax over logits built here from the
+    tagged planes, the plane of key t being r for the block and the window and R-1 otherwise.
+    Independent key planes and scale 8 make a wrong plane, a dropped scale or a shifted window an
+    O(1) difference; the last lines check that such mistakes would indeed be seen."""
+    import torch
+    R, W, T, B = 4, 5, 30, 4
+    d = T + B + 2
+    rng = np.random.default_rng(11)
+    Kp = rng.standard_normal((R, 1, T + B, d))
+    Vp = np.broadcast_to(np.eye(T + B, d)[None, None], (R, 1, T + B, d)).copy()
+    q = rng.standard_normal((B, 1, d)) / np.sqrt(d)
+    for r in range(R):
+        for scale in (1.0, 8.0):
+            ob, _ = orc.brute_verify(Kp, Vp, T, B, r, W, 1, q, scale)
+            for j in range(B):
+                p = T + j
+                w = orc.weights(T, j, r, R, W, Kp[r, 0], Kp[R - 1, 0], q[j, 0], scale)
+                assert np.abs(w - ob[j, 0, :p + 1]).max() < 1e-12
+                assert np.abs(ob[j, 0, p + 1:]).max() == 0.0
+                Ksel = np.stack([Kp[r, 0, t] if (t >= T or t >= p - W) else Kp[R - 1, 0, t] for t in range(p + 1)])
+                ref = torch.softmax(scale * torch.from_numpy(Ksel @ q[j, 0]), dim=0).numpy()
+                assert np.abs(w - ref).max() < 1e-12
+                if r < R - 1 and scale == 1.0:   # every key at the deepest plane instead
+                    wrong_plane = orc.weights(T, j, R - 1, R, W, Kp[R - 1, 0], Kp[R - 1, 0], q[j, 0], scale)
+                    assert np.abs(wrong_plane - ref).sum() > 0.05
+                if scale != 1.0:
+                    no_scale = torch.softmax(torch.from_numpy(Ksel @ q[j, 0]), dim=0).numpy()
+                    assert np.abs(w - no_scale).sum() > 0.05
+
+
 # ---------------------------------------------------------------- plane counts (closed form)
 def _count_closed_form(T, j, r, R, W, mode):
     """Keys read at plane r by query p = T + j: [min(T, max(0, p - W)), p] (query window) or

@@ -13,7 +13,10 @@ import ctypes
 import pytest
 import torch
 
-from harness import check_close, check_lse
+import numpy as np
+
+from harness import Case, check_close, check_lse, dev_to_bits
+from oracle import ripe_oracle as orc
 from self_speculative_decode_b200 import ripe
 from self_speculative_decode_b200.ripe import CacheView, RipeCache, RipeError
 from self_speculative_decode_b200.synth import PlaneSource
@@ -86,6 +89,22 @@ def test_static_entry_matches_cache_entry(W, g, B, d, cuda_device):
                 torch.cuda.synchronize()
                 check_close(out, ref.double().cpu().numpy(), f"static layer {layer} loop {r}")
                 check_lse(lse, lse_ref.double().cpu().numpy())
+    # one call against the CPU oracle directly (layer 1, loop R-2: window, block and deepest keys)
+    layer, r = 1, R - 2
+    oc = orc.OracleCache(N, 1, kvH, d, R, W, max_T)
+    for pl in range(R):
+        oc.load_prefix(0, pl, T, dev_to_bits(PK[layer][pl]), dev_to_bits(PV[layer][pl]))
+    for pl in range(R):
+        kb = torch.stack([PK[layer][pl][n, :, T[n]:T[n] + B].permute(1, 0, 2) for n in range(N)])
+        vb = torch.stack([PV[layer][pl][n, :, T[n]:T[n] + B].permute(1, 0, 2) for n in range(N)])
+        oc.append(0, pl, dev_to_bits(kb), dev_to_bits(vb))
+    q = src[layer].queries(r, B, Hq)
+    out = torch.empty((N, B, Hq, d), dtype=torch.bfloat16, device=cuda_device)
+    lse = torch.empty((N, B, Hq), dtype=torch.float32, device=cuda_device)
+    ripe.ripe_verify_attn_static(view, layer, r, q.data_ptr(), out.data_ptr(), lse.data_ptr(), 1.0, err.data_ptr())
+    ro, rl = oc.verify(0, r, np.ascontiguousarray(dev_to_bits(q)), g)
+    check_close(out, ro, "static vs oracle")
+    check_lse(lse, rl)
     assert int(err.item()) == 0
     assert cache.device_error() == 0
     cache.close()
@@ -98,3 +117,40 @@ def test_static_entry_rejects_problems_beyond_its_scratch(cuda_device):
     with pytest.raises(RipeError) as e:
         ripe.ripe_verify_attn_static(big, 0, 0, 1 << 20, 1 << 20)
     assert e.value.status == ripe.RIPE_ESCRATCH
+
+
+def test_static_call_leaves_larger_caches_usable(cuda_device):
+    """A cache of batch 16 and one of batch 1 are live; an allocation-free call at batch 1 runs;
+    the batch-16 cache then still verifies within tolerance of the CPU oracle, and every call
+    returns RIPE_OK.  (A launch asks for shared memory that grows with the batch: no call may
+    lower the kernels' limit below what a live cache of a larger batch needs.)"""
+    N, kvH, g, d, R, W, B = 1, 2, 2, 96, 3, 16, 4
+    T16 = [130 + 37 * n for n in range(16)]
+    big = Case(N=16, L=1, Hq=kvH * g, kvH=kvH, d=d, R=R, T=T16, W=W, B=B, seed=14, independent=True,
+               oracle_seqs=[0, 9, 15])
+    small = Case(N=1, L=1, Hq=kvH * g, kvH=kvH, d=d, R=R, T=[300], W=W, B=B, seed=15, independent=True,
+                 backend="torch")
+    # the allocation-free view of a batch-1 cache with the same planes as ``small`` (same generator
+    # arguments: seed, layer 0, length, rho, tagged planes, torch backend)
+    T, max_T = [300], 300 + B
+    src = PlaneSource(N, kvH, d, R, max_T, 0.88, 15, independent=True, backend="torch", device=cuda_device)
+    PK = [src.plane(pl, "K") for pl in range(R)]
+    PV = [src.plane(pl, "V") for pl in range(R)]
+    kd, kr = _layout(PK, T, W, B, R, max_T, B)
+    vd, vr = _layout(PV, T, W, B, R, max_T, B)
+    lengths = torch.tensor(T, dtype=torch.int32, device=cuda_device)
+    err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    view = CacheView(batch=N, layers=1, q_heads=kvH * g, kv_heads=kvH, head_dim=d, loops=R, window=W,
+                     max_T=max_T, max_B=B, window_mode=0, block_len=B, k_deep=kd.data_ptr(), v_deep=vd.data_ptr(),
+                     k_ring=kr.data_ptr(), v_ring=vr.data_ptr(), lengths=lengths.data_ptr())
+    for r in range(R):
+        q = torch.randn((N, B, kvH * g, d), device=cuda_device).div(d ** 0.5).to(torch.bfloat16)
+        out = torch.empty_like(q)
+        ripe.ripe_verify_attn_static(view, 0, r, q.data_ptr(), out.data_ptr(), None, 1.0, err.data_ptr())
+        ref = small.gpu.verify_attn(0, r, q)
+        torch.cuda.synchronize()
+        check_close(out, ref.double().cpu().numpy(), f"static batch 1, loop {r}")
+        big.check(0, r)          # raises RipeError (RIPE_ECUDA) if its launch were refused
+    assert int(err.item()) == 0
+    small.close()
+    big.close()
