@@ -10,10 +10,10 @@
  *   Self-Speculative Decoding in Looped Language Models" (arXiv 2610.34436),
  *   abstract, first, fourth and fifth sentences.
  * Accept / rollback of a draft block follows the draft-then-verify scheme as
- * described in the WaveFront Decoding write-up (rit.work blog, section "the
- * draft and the check pass through the model at once"): the verified prefix of
- * the block is kept, the full-depth token replaces the first mismatch, and the
- * drafts after it are discarded.
+ * described in the WaveFront Decoding write-up (rit.work blog, the section on
+ * drafting and checking in one pass): the verified prefix of the block is kept,
+ * the full-depth token replaces the first mismatch, and the drafts after it are
+ * discarded.
  *
  * Conventions for every call:
  *   - Device pointers are plain CUDA device addresses owned by the caller and
@@ -66,7 +66,18 @@ enum ripe_window_mode { RIPE_WINDOW_QUERY_RELATIVE = 0, RIPE_WINDOW_CACHE_RELATI
 enum ripe_device_error {
     RIPE_DEVERR_WAIT_TIMEOUT = 1u, /* a kernel gave up waiting for its own copies */
     RIPE_DEVERR_CAPACITY = 2u,     /* a kernel saw T + B > max_T and skipped its work */
-    RIPE_DEVERR_ACCEPT = 4u        /* a device-side accepted length was outside [0, B] */
+    RIPE_DEVERR_ACCEPT = 4u,       /* a device-side accepted length was outside [0, B] */
+    RIPE_DEVERR_BOUNDS = 8u        /* debug builds: a tile, slot or scratch index fell outside its
+                                      region (the access is still made in bounds: TMA clips it) */
+};
+
+/* Bits of ripe_build_info(). */
+enum ripe_build_flags {
+    RIPE_BUILD_DEBUG = 1 /* built with -DRIPE_DEBUG: device-side index checks set RIPE_DEVERR_BOUNDS,
+                            and every commit fills the ring slots and deepest-plane rows that hold
+                            no live position with the largest finite bf16 (0x7F7F), so that a read
+                            of a dead slot with non-zero weight shows up as a wrong (huge or
+                            non-finite) output instead of a plausible stale value */
 };
 
 typedef struct ripe_stats {
@@ -269,6 +280,9 @@ int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream);
  * host threads) race on the array and must be serialised by the caller.
  * The view's buffers must stay valid until the work enqueued on `stream` has finished.
  * `device_error` (device uint32, optional) receives RIPE_DEVERR_* bits; the caller clears it.
+ * Pass it: with NULL the bits go to a word inside the static array that the next call clears,
+ * so a kernel that skipped its work (RIPE_DEVERR_CAPACITY: T + block_len > max_T for some
+ * sequence; RIPE_DEVERR_WAIT_TIMEOUT) leaves out and lse unwritten without any trace.
  */
 #define RIPE_STATIC_SCRATCH_BYTES (4u << 20)
 
@@ -286,6 +300,9 @@ typedef struct ripe_cache_view {
 
 int ripe_verify_attn_static(const ripe_cache_view *view, int layer, int r, const void *q, void *out,
                             float *lse, float scale, uint32_t *device_error, void *stream);
+
+/* How the library was built: RIPE_BUILD_* bits (no device work, no arguments). */
+int ripe_build_info(void);
 
 /* Number of kernel launches the library has enqueued since the cache was allocated. */
 int64_t ripe_launch_count(const ripe_cache_t *c);

@@ -55,7 +55,7 @@ void release(ripe_cache *c) {
 }
 
 template <typename T>
-bool dalloc(T **p, size_t bytes, int64_t *acct) {
+bool dalloc(T **p, size_t bytes, int64_t *acct, int fill = 0) {
     *p = nullptr;
     if (bytes == 0) return true;
     if (cudaMalloc(reinterpret_cast<void **>(p), bytes) != cudaSuccess) {
@@ -64,7 +64,7 @@ bool dalloc(T **p, size_t bytes, int64_t *acct) {
         return false;
     }
     *acct += static_cast<int64_t>(bytes);
-    return cudaMemset(*p, 0, bytes) == cudaSuccess;
+    return cudaMemset(*p, fill, bytes) == cudaSuccess;
 }
 
 // Calls run with the cache's device current.
@@ -112,6 +112,7 @@ const char *ripe_strerror(int status) {
 
 int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_dim, int loops, int window,
                      int max_T, int max_B, int window_mode, ripe_cache_t **out) {
+    const NvtxRange nvtx_range("ripe_cache_alloc");
     if (!out) return RIPE_EINVAL;
     *out = nullptr;
     if (batch < 1 || batch > kMaxBatch || layers < 1 || q_heads < 1 || kv_heads < 1 || q_heads % kv_heads ||
@@ -137,6 +138,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     c->drafted.assign(static_cast<size_t>(layers) * loops, 0);
     c->prefix_set = false;
     c->synced = true;
+    c->lengths_dirty = true;
     c->kv_bytes = c->scratch_bytes = 0;
     c->launches = 0;
 
@@ -153,8 +155,11 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
     if (c->part_rows > 16 && c->part_rows < 32) c->part_rows = 32;
     if (c->part_rows > 32) c->part_rows = 64;
     c->part_slots = c->num_sms + batch * kv_heads;
-    bool ok = dalloc(&c->Kd, deep_elems * 2, &c->kv_bytes) && dalloc(&c->Vd, deep_elems * 2, &c->kv_bytes) &&
-              dalloc(&c->Kw, ring_elems * 2, &c->kv_bytes) && dalloc(&c->Vw, ring_elems * 2, &c->kv_bytes) &&
+    const int kv_fill = kDebug ? kPoisonByte : 0;  // debug builds: no row holds a position yet
+    bool ok = dalloc(&c->Kd, deep_elems * 2, &c->kv_bytes, kv_fill) &&
+              dalloc(&c->Vd, deep_elems * 2, &c->kv_bytes, kv_fill) &&
+              dalloc(&c->Kw, ring_elems * 2, &c->kv_bytes, kv_fill) &&
+              dalloc(&c->Vw, ring_elems * 2, &c->kv_bytes, kv_fill) &&
               dalloc(&c->T_dev, batch * sizeof(int32_t), &c->scratch_bytes) &&
               dalloc(&c->err_dev, sizeof(uint32_t), &c->scratch_bytes) &&
               dalloc(&c->part_o, static_cast<size_t>(c->part_slots) * c->part_rows * d * sizeof(float),
@@ -186,6 +191,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
 }
 
 int ripe_cache_free(ripe_cache_t *c) {
+    const NvtxRange nvtx_range("ripe_cache_free");
     if (!c) return RIPE_OK;
     DeviceGuard g(c->device);
     cudaDeviceSynchronize();
@@ -195,6 +201,7 @@ int ripe_cache_free(ripe_cache_t *c) {
 
 int ripe_load_prefix(ripe_cache_t *c, int layer, int plane, const int32_t *T, const void *k, const void *v,
                      int64_t ld_t, void *stream) {
+    const NvtxRange nvtx_range("ripe_load_prefix");
     if (!c || !T || !k || !v || layer < 0 || layer >= c->L || plane < 0 || plane >= c->R) return RIPE_EINVAL;
     if (c->B_cur != 0 || !c->synced || any_drafted(c)) return RIPE_ESTATE;
     int Tmax = 0;
@@ -217,6 +224,7 @@ int ripe_load_prefix(ripe_cache_t *c, int layer, int plane, const int32_t *T, co
 }
 
 int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, const void *v, void *stream) {
+    const NvtxRange nvtx_range("ripe_append_block");
     if (!c || !k || !v || layer < 0 || layer >= c->L || r < 0 || r >= c->R || B < 1 || B > c->max_B)
         return RIPE_EINVAL;
     if (c->B_cur != 0 && B != c->B_cur) return RIPE_EINVAL;
@@ -234,6 +242,7 @@ int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, c
 
 int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out, float *lse, float scale,
                      void *stream) {
+    const NvtxRange nvtx_range("ripe_verify_attn");
     if (!c || !q || !out || layer < 0 || layer >= c->L || r < 0 || r >= c->R) return RIPE_EINVAL;
     if (c->B_cur == 0 || !c->appended[static_cast<size_t>(layer) * c->R + r]) return RIPE_ESTATE;
     DeviceGuard g(c->device);
@@ -243,6 +252,7 @@ int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out
 
 int ripe_append_verify(ripe_cache_t *c, int layer, int r, int B, const void *k, const void *v, const void *q,
                        void *out, float *lse, float scale, void *stream) {
+    const NvtxRange nvtx_range("ripe_append_verify");
     if (!c || !k || !v || !q || !out || layer < 0 || layer >= c->L || r < 0 || r >= c->R || B < 1 ||
         B > c->max_B)
         return RIPE_EINVAL;
@@ -284,17 +294,20 @@ static int draft_step(ripe_cache_t *c, int layer, int r, int j, int sink, int wi
 
 int ripe_draft_attn(ripe_cache_t *c, int layer, int r, int j, const void *k, const void *v, const void *q,
                     void *out, float *lse, float scale, void *stream) {
+    const NvtxRange nvtx_range("ripe_draft_attn");
     return draft_step(c, layer, r, j, 0, -1, k, v, q, out, lse, scale, stream);
 }
 
 int ripe_draft_attn_window(ripe_cache_t *c, int layer, int r, int j, int sink, int window, const void *k,
                            const void *v, const void *q, void *out, float *lse, float scale, void *stream) {
+    const NvtxRange nvtx_range("ripe_draft_attn_window");
     if (sink < 0 || window < 0) return RIPE_EINVAL;
     return draft_step(c, layer, r, j, sink, window, k, v, q, out, lse, scale, stream);
 }
 
 int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                           float *lse, float scale, void *stream) {
+    const NvtxRange nvtx_range("ripe_verify_attn_wave");
     if (!c || !loop_of_position || !q || !out || layer < 0 || layer >= c->L) return RIPE_EINVAL;
     if (c->B_cur == 0) return RIPE_ESTATE;
     for (int j = 0; j < c->B_cur; ++j) {
@@ -308,6 +321,7 @@ int ripe_verify_attn_wave(ripe_cache_t *c, int layer, const int32_t *loop_of_pos
 }
 
 int ripe_commit(ripe_cache_t *c, const int32_t *accepted_len, void *stream) {
+    const NvtxRange nvtx_range("ripe_commit");
     if (!c || !accepted_len) return RIPE_EINVAL;
     if (c->B_cur == 0 || !all_appended(c)) return RIPE_ESTATE;
     for (int n = 0; n < c->N; ++n)
@@ -324,6 +338,7 @@ int ripe_commit(ripe_cache_t *c, const int32_t *accepted_len, void *stream) {
 }
 
 int ripe_commit_device(ripe_cache_t *c, const int32_t *accepted_len, void *stream) {
+    const NvtxRange nvtx_range("ripe_commit_device");
     if (!c || !accepted_len) return RIPE_EINVAL;
     if (c->B_cur == 0 || !all_appended(c)) return RIPE_ESTATE;
     DeviceGuard g(c->device);
@@ -339,6 +354,7 @@ int ripe_commit_device(ripe_cache_t *c, const int32_t *accepted_len, void *strea
 }
 
 int ripe_sync_lengths(ripe_cache_t *c, int32_t *T_out, void *stream) {
+    const NvtxRange nvtx_range("ripe_sync_lengths");
     if (!c) return RIPE_EINVAL;
     DeviceGuard g(c->device);
     if (!g.ok) return RIPE_ECUDA;
@@ -372,6 +388,7 @@ int ripe_cache_stats(const ripe_cache_t *c, ripe_stats *st) {
 
 int ripe_cache_export(ripe_cache_t *c, int n, int layer, void *k_out, void *v_out, uint8_t *plane_present,
                       void *stream) {
+    const NvtxRange nvtx_range("ripe_cache_export");
     if (!c || !k_out || !v_out || !plane_present || n < 0 || n >= c->N || layer < 0 || layer >= c->L)
         return RIPE_EINVAL;
     if (!c->synced) return RIPE_ESTATE;
@@ -381,6 +398,7 @@ int ripe_cache_export(ripe_cache_t *c, int n, int layer, void *k_out, void *v_ou
 }
 
 int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream) {
+    const NvtxRange nvtx_range("ripe_get_device_error");
     if (!c || !err_out) return RIPE_EINVAL;
     DeviceGuard g(c->device);
     if (!g.ok) return RIPE_ECUDA;
@@ -401,5 +419,7 @@ int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream) {
 }
 
 int64_t ripe_launch_count(const ripe_cache_t *c) { return c ? c->launches : -1; }
+
+int ripe_build_info(void) { return kDebug ? RIPE_BUILD_DEBUG : 0; }
 
 }  // extern "C"

@@ -8,9 +8,26 @@
 
 #include <vector>
 
+#ifndef RIPE_NO_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 #include "ripe.h"
 
 namespace ripe {
+
+// A named range around each C-ABI call for profilers (NVTX, header-only; a branch on a null
+// function pointer when no tool is attached).  -DRIPE_NO_NVTX compiles it out.
+struct NvtxRange {
+#ifndef RIPE_NO_NVTX
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+#else
+    explicit NvtxRange(const char *) {}
+#endif
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 constexpr int kMaxBatch = 1024;   // sequences per cache (accepted lengths travel as kernel parameters)
 constexpr int kMaxLoops = 256;    // R
@@ -20,6 +37,14 @@ constexpr int kBoxBytes = kTileRows * 64;  // one box slot in shared memory (4 K
 constexpr int kStages = 4;        // TMA pipeline depth of the verify kernel
 constexpr int kMaxQueryRows = 64; // B * (Hq / kvH) per key/value head
 constexpr int kMaxDevices = 64;   // devices a process may drive (per-device set-up tables)
+// debug builds: bf16 bits written into key/value rows that hold no live position (the largest
+// finite value: a masked read multiplies it by 0, any weighted read overflows the output)
+constexpr int kPoisonByte = 0x7F;
+#ifdef RIPE_DEBUG
+constexpr bool kDebug = true;
+#else
+constexpr bool kDebug = false;
+#endif
 
 // Bounded waits: a kernel that does not see its copies land within this time records
 // RIPE_DEVERR_WAIT_TIMEOUT and stops (it never traps).
@@ -55,6 +80,9 @@ struct ripe_cache {
     std::vector<uint8_t> appended;  // [L][R] planes of the block appended
     std::vector<int> drafted;       // [L][R] draft positions written at each plane (before the block)
     bool prefix_set, synced;
+    // the last launch on this cache wrote the lengths T or the deepest-plane region (commit with
+    // eviction, prefix load): the next verify waits for it before reading either
+    bool lengths_dirty;
     int64_t kv_bytes, scratch_bytes;
     int64_t launches;
 };
@@ -429,6 +457,7 @@ int launch_load_prefix(ripe_cache *c, int layer, int plane, const int32_t *T, co
                        const void *v, int64_t ld_t, cudaStream_t s);
 int launch_export(ripe_cache *c, int n, int layer, void *k_out, void *v_out, uint8_t *present,
                   cudaStream_t s);
+int launch_poison(ripe_cache *c, cudaStream_t s);  // debug builds: refill dead rows after a commit
 // Raise the verify kernels' dynamic shared-memory limit on `device` (which must be current) to
 // what the largest batch needs; once per device, thread-safe.
 int ensure_verify_attributes(int device);
@@ -446,6 +475,8 @@ struct RawVerify {
     PlanArgs plan;
     int N, kvH, g, Hq, d, layer, grid, has_deep;
     int device, num_sms;
+    int dbg_deep_rows;
+    long long dbg_deep_pages, dbg_ring_pages;
     float scale;
 };
 int launch_verify_raw(const RawVerify &rv, cudaStream_t s);

@@ -62,6 +62,7 @@ int launch_append(ripe_cache *c, int layer, int r, int B, const void *k, const v
                static_cast<const int32_t *>(c->T_dev), c->err_dev, c->N, B, c->kvH, d8, c->R, c->ring_slots, layer,
                r, c->max_T);
     c->launches += 1;
+    c->lengths_dirty = false;
     return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 
@@ -100,7 +101,10 @@ __global__ void ripe_evict_kernel(uint4 *__restrict__ Kd, uint4 *__restrict__ Vd
         const int rest = idx / d8;
         const int kh = rest % kvH;
         const int t = lo + rest / kvH;
-        if (t >= deep_rows) continue;  // cannot happen while T + B <= max_T
+        if (t >= deep_rows) {  // cannot happen while T + B <= max_T
+            if (kDebug) atomicOr(err, RIPE_DEVERR_BOUNDS);
+            continue;
+        }
         const size_t src = ring_row(layer, n, R - 1, kh, t % S, N, R, kvH, S) * d8 + c8;
         const size_t dst = deep_row(layer, n, kh, t, N, kvH, deep_rows) * d8 + c8;
         Kd[dst] = Kw[src];
@@ -116,6 +120,7 @@ __global__ void ripe_commit_lengths_kernel(int32_t *T, const HostIntArray acc_h,
 }
 
 int launch_commit(ripe_cache *c, const int32_t *acc_host, const int32_t *acc_dev, cudaStream_t s) {
+    c->lengths_dirty = true;
     HostIntArray ah;
     for (int n = 0; n < c->N; ++n) ah.v[n] = acc_host ? acc_host[n] : 0;
     const int d8 = c->d / 8;
@@ -133,6 +138,61 @@ int launch_commit(ripe_cache *c, const int32_t *acc_host, const int32_t *acc_dev
     }
     launch_pdl(ripe_commit_lengths_kernel, dim3(1), dim3(256), 0, s, c->T_dev, ah, acc_dev, c->err_dev, c->N,
                c->B_cur);
+    c->launches += 1;
+    c->lengths_dirty = true;
+    if (cudaGetLastError() != cudaSuccess) return RIPE_ECUDA;
+    return kDebug ? launch_poison(c, s) : RIPE_OK;
+}
+
+// ---------------------------------------------------------------- dead-row poisoning (debug builds)
+// After a commit the live rows are: ring slots holding positions [max(0, T - W), T) (every plane)
+// and deepest-plane rows [0, max(0, T - W)).  Every other ring slot (rolled-back drafts, positions
+// that left the window) and deepest-plane row (not evicted yet) gets the poison pattern, so a kernel
+// that reads one with non-zero weight produces a wrong output that the parity tests catch.
+__global__ void ripe_poison_kernel(uint4 *__restrict__ Kd, uint4 *__restrict__ Vd, uint4 *__restrict__ Kw,
+                                   uint4 *__restrict__ Vw, const int32_t *__restrict__ T, int L, int N, int R,
+                                   int kvH, int d8, int S, int W, int deep_rows) {
+    const uint32_t pw = kPoisonByte * 0x01010101u;
+    const uint4 poison = make_uint4(pw, pw, pw, pw);
+    const size_t ring_rows = static_cast<size_t>(L) * N * R * kvH * S;
+    const size_t deep_total = static_cast<size_t>(L) * N * kvH * deep_rows;
+    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+    for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < (ring_rows + deep_total) * d8;
+         idx += stride) {
+        const size_t row = idx / d8;
+        if (row < ring_rows) {
+            const int slot = static_cast<int>(row % S);
+            const size_t rest = row / S / kvH / R;  // layer * N + n
+            const int n = static_cast<int>(rest % N);
+            const int Tn = T[n];
+            const int lo = Tn - W > 0 ? Tn - W : 0;
+            const int off = ((slot - lo % S) + S) % S;  // slot of position lo + off
+            if (off < Tn - lo) continue;                // a live window position
+            Kw[idx] = poison;
+            Vw[idx] = poison;
+        } else {
+            const size_t drow = row - ring_rows;
+            const int t = static_cast<int>(drow % deep_rows);
+            const int n = static_cast<int>((drow / deep_rows / kvH) % N);
+            const int lo = T[n] - W > 0 ? T[n] - W : 0;
+            if (t < lo) continue;                       // evicted into the deepest-plane region
+            const size_t e = idx - ring_rows * d8;
+            Kd[e] = poison;
+            Vd[e] = poison;
+        }
+    }
+}
+
+int launch_poison(ripe_cache *c, cudaStream_t s) {
+    const int d8 = c->d / 8;
+    const size_t rows = static_cast<size_t>(c->L) * c->N * c->kvH * (static_cast<size_t>(c->R) * c->ring_slots +
+                                                                      static_cast<size_t>(c->deep_rows));
+    size_t blocks = (rows * d8 + 255) / 256;
+    if (blocks > static_cast<size_t>(8 * c->num_sms)) blocks = 8 * c->num_sms;
+    ripe_poison_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(
+        reinterpret_cast<uint4 *>(c->Kd), reinterpret_cast<uint4 *>(c->Vd), reinterpret_cast<uint4 *>(c->Kw),
+        reinterpret_cast<uint4 *>(c->Vw), c->T_dev, c->L, c->N, c->R, c->kvH, d8, c->ring_slots, c->W,
+        c->deep_rows);
     c->launches += 1;
     return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
@@ -190,6 +250,7 @@ int launch_load_prefix(ripe_cache *c, int layer, int plane, const int32_t *T, co
         th, c->N, c->kvH, d8, c->R, c->ring_slots, c->W, c->deep_rows, layer, plane, Tmax > 0 ? Tmax : 1,
         static_cast<long long>(ld_t));
     c->launches += 1;
+    c->lengths_dirty = true;
     return cudaGetLastError() == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 

@@ -85,6 +85,7 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int r, const void *q, void *out,
                                        float *lse, float scale, uint32_t *device_error, void *stream) {
     using namespace ripe;
+    const NvtxRange nvtx_range("ripe_verify_attn_static");
     if (!v || !q || !out) return RIPE_EINVAL;
     const int N = v->batch, L = v->layers, Hq = v->q_heads, kvH = v->kv_heads, d = v->head_dim, R = v->loops;
     if (N < 1 || N > kMaxBatch || L < 1 || Hq < 1 || kvH < 1 || Hq % kvH || (d != 64 && d != 96 && d != 128) ||
@@ -168,6 +169,9 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.grid = grid;
     rv.device = dev;
     rv.num_sms = ds->num_sms;
+    rv.dbg_deep_rows = deep_rows;
+    rv.dbg_deep_pages = deep_pages;
+    rv.dbg_ring_pages = ring_pages;
     rv.has_deep = deep_rows > 0 ? 1 : 0;
     rv.scale = scale;
     const int ls = launch_verify_raw(rv, s);

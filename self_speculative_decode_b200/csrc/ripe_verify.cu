@@ -57,11 +57,18 @@ struct VerifyArgs {
     // CTA holding the second piece sends its partial to the first through distributed shared memory
     int xpair;
     int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
+    // early start: the previous launch on the stream writes neither the lengths T nor the
+    // deepest-plane region, so both are read, and deepest-plane tiles streamed, before waiting for
+    // it (programmatic dependent launch); everything else waits
+    int early;
     float scale_log2;
     // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
     const uint4 *blk_k, *blk_v;
     uint4 *ring_k, *ring_v;
     int max_T;
+    // region sizes for the index checks of debug builds
+    int dbg_deep_rows, dbg_part_slots;
+    long long dbg_deep_pages, dbg_ring_pages;
 };
 
 constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
@@ -297,7 +304,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         for (int i = tid; i < NS * C::STAGE_BYTES / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
     }
     // ---- per-sequence tile counts and their prefix sums (T is written by earlier kernels)
-    pdl_wait();
+    if (!a.early) pdl_wait();
     int total, chunk, pieces;  // pieces 0: contiguous chunks of the whole tile list
     int tot_head = 0;          // tiles per (sequence, kv head) in piece mode
     SeqGeom sg1 = {};          // the sequence's geometry when N == 1
@@ -368,7 +375,10 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         g_begin = blockIdx.x * chunk;
         g_end = min(total, g_begin + chunk);
     }
-    if (g_begin >= g_end) return;
+    if (g_begin >= g_end) {
+        if (a.early) pdl_wait();  // the launch completes only after its predecessor
+        return;
+    }
     const int ntiles = g_end - g_begin;
     // (sequence, kv head) pairs of this CTA's first and last tiles
     const int P_first = pieces ? head : pair_of(cum, N, kvH, g_begin);
@@ -385,6 +395,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         if (warp == C::NCW + 1) {
             // the copy warp: write the draft block's rows that this CTA's tiles read into the
             // ring, fence them for the TMA (async proxy), release the producer
+            if (a.early) pdl_wait();  // the caller's block rows and the ring slots they replace
             fused_block_copy<D>(a, cum, Ts, g_begin, g_end, lane, 32);
             asm volatile("fence.proxy.async.global;" ::: "memory");
             __syncwarp();
@@ -394,6 +405,17 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     }
     if (warp == C::NCW) {
         // ================================================================ producer (one thread)
+        if (lane != 0 && a.early) {
+            // the other lanes bring the first pair's query rows into L2 while the previous launch
+            // finishes (the consumers load them once it has)
+            const int n0 = P_first / kvH, kh0 = P_first - n0 * kvH;
+            for (int i = lane - 1; i < a.Mq; i += 31) {
+                const int j = i / a.g, hg = i - j * a.g;
+                const char *row = reinterpret_cast<const char *>(
+                    a.q + ((static_cast<size_t>(n0) * a.qB + j) * a.Hq + kh0 * a.g + hg) * D);
+                for (int off = 0; off < D * 2; off += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(row + off));
+            }
+        }
         if (lane == 0) {
             int n, kh, lt;
             SeqGeom sg;
@@ -412,6 +434,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             const int P0 = P_first;
             int i = 0;
             bool ok = true;
+            bool waited = !a.early;
             // with a fused append, the tiles holding the rows this launch writes wait until the
             // copy warp has written them: the loop below runs in two phases, up to the first such
             // tile of the chunk and from it, and stays free of a per-tile check
@@ -426,11 +449,24 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 }
                 const Tile t = tile_at(sg, lt, pa);
                 const bool deep = t.kind == kDeep;
+                if (!waited && !deep) {  // ring rows: the previous launch may be writing the block
+                    pdl_wait();
+                    waited = true;
+                }
                 const int rows = deep ? pa.deep_box : pa.ring_box;
                 const CUtensorMap *mk = deep ? &tmKd : &tmKw;
                 const CUtensorMap *mv = deep ? &tmVd : &tmVw;
                 const int z = deep ? ((a.layer * N + n) * kvH + kh)
                                    : (((a.layer * N + n) * a.R + t.plane) * kvH + kh);
+                if constexpr (kDebug) {  // the tile lies inside its region and inside the plan
+                    const bool bad =
+                        t.cnt < 1 || t.cnt > rows ||
+                        (deep ? (t.t0 < 0 || t.t0 + t.cnt > sg.D || sg.D > a.dbg_deep_rows || z >= a.dbg_deep_pages)
+                              : (t.y < 0 || t.y + t.cnt > pa.ring_slots || t.t0 < sg.D ||
+                                 t.t0 + t.cnt > (t.kind == kDual ? sg.T : sg.T + a.B) || z >= a.dbg_ring_pages ||
+                                 (t.y - (t.t0 % pa.ring_slots) + pa.ring_slots) % pa.ring_slots != 0));
+                    if (bad) atomicOr(a.err, RIPE_DEVERR_BOUNDS);
+                }
                 TileDesc &dsc = sdesc[s];
                 dsc.pair = n * kvH + kh; dsc.n = n; dsc.kh = kh; dsc.T = sg.T;
                 dsc.kind = t.kind; dsc.t0 = t.t0; dsc.cnt = t.cnt; dsc.plane = t.plane;
@@ -701,6 +737,10 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 op[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
                 if (c0 == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
             } else {
+                if (kDebug && static_cast<int>(blockIdx.x) + p >= a.dbg_part_slots) {
+                    atomicOr(a.err, RIPE_DEVERR_BOUNDS);
+                    continue;
+                }
                 const size_t prow = (static_cast<size_t>(blockIdx.x) + p) * C::ROWS + i;
                 *reinterpret_cast<float4 *>(&a.part_o[prow * D + c0]) = acc;
                 if (c0 == 0) {
@@ -898,9 +938,14 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         }
     };
 
+    // ring tiles can take the mask-free path only when every query is at the tile's loop and no
+    // draft window cuts keys out
+    const bool ring_all_visible = pa.nloops == 1 && pa.dwin < 0;
     reset_state();
-    // the first pair's queries: loaded while its first tile is still in flight
+    // the first pair's queries: loaded while its first tile is still in flight (with an early
+    // start, once the previous launch has finished: the caller may be writing them)
     st_pair = P_first;
+    if (a.early) pdl_wait();
     load_q(P_first / kvH, P_first - (P_first / kvH) * kvH);
     for (int i = tg; i < ntiles; i += TG) {
         const int s = i % NS;
@@ -920,7 +965,15 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             reset_state();
             load_q(dsc.n, dsc.kh);
         }
-        if (dsc.kind == kDeep && dsc.cnt == kTileRows)
+        // mask-free: a full deepest-plane tile, or a full ring tile that every query of the call
+        // sees whole (one loop; every key before the first query and inside the last query's
+        // window, as for the full cache and windows wider than the prefix)
+        const bool full_view =
+            dsc.cnt == kTileRows &&
+            (dsc.kind == kDeep ||
+             (dsc.kind == kRing && ring_all_visible && dsc.t0 + kTileRows - 1 <= dsc.T + a.j0 &&
+              (pa.mode_eff != 0 || dsc.t0 >= dsc.T + a.j0 + a.qB - 1 - pa.W)));
+        if (full_view)
             compute(dsc, s, std::integral_constant<bool, true>());
         else
             compute(dsc, s, std::integral_constant<bool, false>());
@@ -1103,6 +1156,11 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.Mq = rv.plan.B * rv.g;
     a.min_chunk = RIPE_MIN_CHUNK;
     a.has_deep = rv.has_deep;
+    a.dbg_deep_rows = rv.dbg_deep_rows;
+    a.dbg_part_slots = rv.grid + rv.N * rv.kvH;
+    a.dbg_deep_pages = rv.dbg_deep_pages;
+    a.dbg_ring_pages = rv.dbg_ring_pages;
+    a.early = 0;  // the caller's own kernels may write the cache buffers
     a.scale_log2 = rv.scale * 1.4426950408889634f;
     const LaunchTarget t = {&rv.tmKd, &rv.tmVd, &rv.tmKw, &rv.tmVw, rv.device, rv.num_sms, rv.N};
     if (rv.d != 64 && rv.d != 96 && rv.d != 128) return RIPE_EINVAL;
@@ -1199,6 +1257,11 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
     a.Mq = a.qB * c->g;
     a.min_chunk = RIPE_MIN_CHUNK;  // bounds the number of partials of one (sequence, kv head)
     a.has_deep = c->deep_rows > 0 ? 1 : 0;
+    a.dbg_deep_rows = c->deep_rows;
+    a.dbg_part_slots = c->part_slots;
+    a.dbg_deep_pages = static_cast<long long>(c->L) * c->N * c->kvH;
+    a.dbg_ring_pages = static_cast<long long>(c->L) * c->N * c->R * c->kvH;
+    a.early = c->lengths_dirty ? 0 : 1;
     a.scale_log2 = scale * 1.4426950408889634f;
     const int qc = qcfg_of(a.Mq);
 
@@ -1215,6 +1278,7 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
     const LaunchTarget t = {&c->tm_Kd, &c->tm_Vd, &c->tm_Kw, &c->tm_Vw, c->device, c->num_sms, c->N};
     const cudaError_t e = launch_any(c->d, qc, t, grid, a, s);
     c->launches += 1;
+    c->lengths_dirty = false;
     return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 

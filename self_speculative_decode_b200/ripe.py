@@ -11,11 +11,14 @@ import ctypes
 import os
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "lib", "libripe.so")
+# the library to load: libripe.so, or another build of the same sources (e.g. the debug build
+# lib/libripe_debug.so) named by the environment variable RIPE_LIBRARY
+LIB_PATH = os.environ.get("RIPE_LIBRARY") or os.path.join(PKG, "lib", "libripe.so")
 
 RIPE_OK, RIPE_EINVAL, RIPE_ENOMEM, RIPE_ECAPACITY, RIPE_ESTATE, RIPE_ECUDA = 0, -1, -2, -3, -4, -5
 RIPE_WINDOW_QUERY_RELATIVE, RIPE_WINDOW_CACHE_RELATIVE = 0, 1
-RIPE_DEVERR_WAIT_TIMEOUT, RIPE_DEVERR_CAPACITY, RIPE_DEVERR_ACCEPT = 1, 2, 4
+RIPE_DEVERR_WAIT_TIMEOUT, RIPE_DEVERR_CAPACITY, RIPE_DEVERR_ACCEPT, RIPE_DEVERR_BOUNDS = 1, 2, 4, 8
+RIPE_BUILD_DEBUG = 1
 
 # exported entry points (kept in step with include/ripe.h; a CPU test checks both)
 EXPORTS = (
@@ -23,7 +26,7 @@ EXPORTS = (
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
     "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave", "ripe_append_verify",
-    "ripe_draft_attn", "ripe_draft_attn_window",
+    "ripe_draft_attn", "ripe_draft_attn_window", "ripe_build_info",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -76,6 +79,7 @@ def lib() -> ctypes.CDLL:
             "ripe_cache_export": ([vp, i, i, vp, vp, vp, vp], i),
             "ripe_get_device_error": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i),
             "ripe_launch_count": ([vp], i64),
+            "ripe_build_info": ([], i),
             "ripe_strerror": ([i], ctypes.c_char_p),
             "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
             "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
@@ -223,6 +227,10 @@ def ripe_verify_attn_static(view, layer, r, q, out, lse=None, scale=1.0, device_
 
 def ripe_launch_count(h):
     return lib().ripe_launch_count(h)
+
+
+def ripe_build_info():
+    return lib().ripe_build_info()
 
 
 # ------------------------------------------------------------------ tensor-level wrapper

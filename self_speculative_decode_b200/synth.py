@@ -8,8 +8,9 @@ Recipe (the pages give no data, only how the planes behave):
   * the deepest plane D of every position is N(0, 1) per element;
   * plane r < R-1 is D + rho**r * eps_r with eps_r ~ N(0, 1) drawn independently
     per plane, separately for keys and values, so the distance to the deepest
-    plane shrinks by rho per loop ("the planes approach the last one
-    geometrically, at 0.88 and 0.81 per loop", RIPE abstract, second sentence);
+    plane shrinks by rho per loop (RIPE abstract, second sentence: the planes
+    converge geometrically on the last one, at 0.88 per loop for Huginn-0125 and
+    0.81 for Raven-Llama);
   * plane R-1 is D itself, the plane that RIPE keeps everywhere;
   * ``independent=True`` draws every plane as its own N(0, 1) sample ("tagged"
     planes): a wrong plane choice then moves an output by O(1) instead of

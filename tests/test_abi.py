@@ -65,3 +65,16 @@ def test_calls_on_a_null_handle_are_rejected():
     assert L.ripe_verify_attn_wave(null, 0, None, null, null, null, 1.0, null) == ripe.RIPE_EINVAL
     assert L.ripe_cache_free(null) == ripe.RIPE_OK
     assert L.ripe_launch_count(null) == -1
+
+
+def test_build_info_tells_the_release_and_debug_builds_apart():
+    """ripe_build_info: 0 for libripe.so; RIPE_BUILD_DEBUG for libripe_debug.so, which exports the
+    same entry points."""
+    from self_speculative_decode_b200 import build
+    if "RIPE_LIBRARY" not in os.environ:
+        assert ripe.ripe_build_info() == 0
+    if not os.path.exists(build.LIB_DEBUG):
+        pytest.skip("debug build not present")
+    dbg = ctypes.CDLL(build.LIB_DEBUG)
+    assert dbg.ripe_build_info() == ripe.RIPE_BUILD_DEBUG
+    assert not [name for name in _declared() if not hasattr(dbg, name)]
