@@ -453,7 +453,7 @@ class L2Flush:
     def __call__(self, i):
         import torch
         self.buf.fill_(float(i))
-        torch.sum(self.buf, out=self.acc)
+        torch.sum(self.buf, dim=0, out=self.acc)
 
 
 def verify_launch_timing(wl, reps, dist_on, peak, cold_calls=32):

@@ -269,7 +269,7 @@ int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream);
  * Its scratch (partial results of the split key ranges and their arrival counters) is one
  * file-scope device array of RIPE_STATIC_SCRATCH_BYTES, which every GPU that loads the
  * library holds until the process exits.  A problem whose scratch would exceed it is rejected
- * with RIPE_ESCRATCH: it needs (S + batch * kv_heads) * rows * (head_dim + 2) * 4 bytes plus
+ * with RIPE_ESCRATCH: it needs (S + batch * kv_heads) * rows * (head_dim + 4) * 4 bytes plus
  * batch * kv_heads * 4, where S is the number of SMs and rows is 8, 16, 32 or 64 (the block
  * length times q_heads / kv_heads, rounded up to one of those).
  *

@@ -164,7 +164,7 @@ int ripe_cache_alloc(int batch, int layers, int q_heads, int kv_heads, int head_
               dalloc(&c->err_dev, sizeof(uint32_t), &c->scratch_bytes) &&
               dalloc(&c->part_o, static_cast<size_t>(c->part_slots) * c->part_rows * d * sizeof(float),
                      &c->scratch_bytes) &&
-              dalloc(&c->part_ml, static_cast<size_t>(c->part_slots) * c->part_rows * 2 * sizeof(float),
+              dalloc(&c->part_ml, static_cast<size_t>(c->part_slots) * c->part_rows * 4 * sizeof(float),
                      &c->scratch_bytes) &&
               dalloc(&c->counters, static_cast<size_t>(batch) * kv_heads * sizeof(int32_t), &c->scratch_bytes);
     if (!ok) {

@@ -70,7 +70,7 @@ struct ripe_cache {
     int32_t *T_dev;          // [N]
     uint32_t *err_dev;       // device error word
     float *part_o;           // [part_slots][part_rows][d]
-    float *part_ml;          // [part_slots][part_rows][2]
+    float *part_ml;          // [part_slots][part_rows][4]: m, l_out, l_lse, -
     int32_t *counters;       // [N * kvH] arrivals per (sequence, kv head), reset by the last arrival
     int part_slots, part_rows;
     CUtensorMap tm_Kd, tm_Vd, tm_Kw, tm_Vw;

@@ -32,59 +32,14 @@
 //     scratch; the last to arrive (atomic counter, no spinning) merges them.
 //   * Every wait is bounded: on timeout the kernel records RIPE_DEVERR_WAIT_TIMEOUT, drains
 //     its own copies in flight and returns without writing further results.
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 #include <type_traits>
 
-#include "ripe_common.cuh"
+#include "ripe_verify.cuh"
 
 namespace ripe {
-
-struct VerifyArgs {
-    const __nv_bfloat16 *q;
-    __nv_bfloat16 *out;
-    float *lse;
-    const int32_t *T;
-    float *part_o;
-    float *part_ml;
-    int32_t *counters;
-    uint32_t *err;
-    PlanArgs plan;
-    int N, kvH, g, Hq, B, R, layer, Mq, min_chunk;
-    // queries: block positions j0 .. j0 + qB - 1 (q, out, lse and the fused block hold qB rows
-    // per sequence); a verification has j0 = 0, qB = B, a draft step j0 = its position, qB = 1
-    int j0, qB;
-    // launched as clusters of 2 CTAs: when each (sequence, kv head) is split into two pieces, the
-    // CTA holding the second piece sends its partial to the first through distributed shared memory
-    int xpair;
-    int has_deep;  // the deepest-plane maps are valid (the full cache has no such region)
-    // early start: the previous launch on the stream writes neither the lengths T nor the
-    // deepest-plane region, so both are read, and deepest-plane tiles streamed, before waiting for
-    // it (programmatic dependent launch); everything else waits
-    int early;
-    float scale_log2;
-    // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
-    const uint4 *blk_k, *blk_v;
-    uint4 *ring_k, *ring_v;
-    int max_T;
-    // region sizes for the index checks of debug builds
-    int dbg_deep_rows, dbg_part_slots;
-    long long dbg_deep_pages, dbg_ring_pages;
-};
-
-constexpr int kSmemLimit = 232448;  // dynamic shared memory per CTA on sm_100
-#ifndef RIPE_MAX_STAGES
-#define RIPE_MAX_STAGES 8               // TMA pipeline depth cap (shared memory sets the rest)
-#endif
-#ifndef RIPE_MAX_STAGES_WIDE
-// head_dim 128 with a single tile group (16-32-query rows per kv head, GQA): 3 stages of 32 KB
-// measured faster than 2 or 4 on B200 (long-context GQA verify: 204 vs 230 / 218 us)
-#define RIPE_MAX_STAGES_WIDE 3
-#endif
-#ifndef RIPE_MIN_CHUNK
-#define RIPE_MIN_CHUNK 4                // at least this many 64-key tiles per CTA
-#endif
-constexpr float kLazyMax = 8.f;     // log2 headroom before the softmax reference moves
-constexpr int kSwitchTiles = 3;     // tiles a CTA may add to its chunk to avoid a mid-stream head switch
 
 // Query-side shapes: NQT 8-query tiles per warp, WR row groups, WK key groups per tile,
 // TG tile groups consuming alternate tiles.
@@ -102,8 +57,9 @@ struct VCfg {
     static constexpr int MERGE_FLOATS = NCW * NQ * DP;
     // receive buffer of the cluster-pair merge: the partner's o [ROWS][D] and (m, l) [ROWS][2]
     static constexpr bool XPAIR = ROWS <= 16;
-    static constexpr int XF = XPAIR ? ROWS * D + 2 * ROWS : 0;
-    static constexpr int MLF = NCW * NQ * 2 + ROWS * (TG * WK + 2) + XF;
+    static constexpr int XF = XPAIR ? ROWS * D + 4 * ROWS : 0;
+    // per (warp, query) and per row: (m, l_out, l_lse, -), see the softmax below
+    static constexpr int MLF = NCW * NQ * 4 + ROWS * (TG * WK + 4) + XF;
     static constexpr int MISC = 1024 /*align*/ + 1024 /*bars, descriptors, flags*/;
     static constexpr int AVAIL = kSmemLimit - MISC - 4 * (MERGE_FLOATS + MLF) - 4 * (2 * kMaxBatch + 2);
     static constexpr int CAP = (D == 128 && TG == 1) ? RIPE_MAX_STAGES_WIDE : RIPE_MAX_STAGES;
@@ -119,64 +75,9 @@ struct VCfg {
 #endif
 };
 
-struct TileDesc {
-    int pair, n, kh, T, kind, t0, cnt, plane;
-};
-
 template <class C>
 __host__ __device__ constexpr int smem_bytes_for(int N) {
     return C::SMEM_FIXED + (2 * N + 2) * 4;
-}
-
-// index of the last sequence whose first tile is <= gt
-__device__ __forceinline__ int seq_of(const int *cum, int N, int gt) {
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (cum[mid] <= gt) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
-
-__device__ __forceinline__ int pair_of(const int *cum, int N, int kvH, int gt) {
-    const int n = seq_of(cum, N, gt);
-    const int tot = (cum[n + 1] - cum[n]) / kvH;
-    return n * kvH + (gt - cum[n]) / tot;
-}
-
-// How a launch of `grid` CTAs cuts `total` tiles (tot0 per (sequence, kv head) when `same`):
-// contiguous chunks of `chunk` tiles (pieces = 0), or, when several CTAs share each head,
-// `pieces` equal pieces of every head, CTA c taking piece c % pieces of head c / pieces.
-// Cuts fall on head boundaries when that costs at most kSwitchTiles tiles per CTA: a CTA then
-// never switches to another head mid-stream.
-__device__ __forceinline__ void choose_chunk(int total, int tot0, bool same, int grid, int N, int kvH, int min_chunk,
-                                             int &chunk, int &pieces) {
-    int ch = cdiv(total, grid);
-    if (ch < min_chunk) ch = min_chunk;
-    pieces = 0;
-    if (same) {
-        if (ch < tot0) {
-            int P = grid / (N * kvH);
-            if (P > tot0 / min_chunk) P = tot0 / min_chunk;
-            if (P >= 1) {
-                const int ca = cdiv(tot0, P);
-                if (ca <= ch + kSwitchTiles) {
-                    ch = ca;
-                    pieces = P;
-                }
-            }
-        } else {
-            const int ca = cdiv(ch, tot0) * tot0;
-            if (ca <= ch + kSwitchTiles) ch = ca;
-        }
-    }
-    chunk = ch;
-}
-
-// Ring tile (index within the pair's list) holding position pos of the single-loop ring [D, T + B).
-__device__ __forceinline__ int ring_tile_of(const SeqGeom &sg, const PlanArgs &pa, int pos) {
-    const int o = pos - sg.D;
-    return sg.nd + (o < sg.ring_first ? o / pa.ring_box : sg.nr1 + (o - sg.ring_first) / pa.ring_box);
 }
 
 // Fused append: the rows of the draft block (positions >= T + j0) inside this CTA's ring tiles
@@ -255,11 +156,11 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                                                 ~static_cast<uintptr_t>(1023));
     uint8_t *stages = base;
     float *mo = reinterpret_cast<float *>(base + NS * C::STAGE_BYTES);   // [NCW][NQ][DP]
-    float *mml = mo + C::MERGE_FLOATS;                                   // [NCW][NQ][2]
-    float *wq = mml + C::NCW * C::NQ * 2;                                // [ROWS][TG*WK] weights
-    float *fin = wq + C::ROWS * TG * WK;                                 // [ROWS][2] final M, L
-    float *xo = fin + C::ROWS * 2;                                       // [ROWS][D] partner's o (XPAIR)
-    float *xml = xo + C::ROWS * D;                                       // [ROWS][2] partner's m, l
+    float *mml = mo + C::MERGE_FLOATS;                                   // [NCW][NQ][4] m, l_out, l_lse
+    float *wq = mml + C::NCW * C::NQ * 4;                                // [ROWS][TG*WK] weights
+    float *fin = wq + C::ROWS * TG * WK;                                 // [ROWS][4] final M, L_out, L_lse
+    float *xo = fin + C::ROWS * 4;                                       // [ROWS][D] partner's o (XPAIR)
+    float *xml = xo + C::ROWS * D;                                       // [ROWS][4] partner's M, L_out, L_lse
     uint64_t *bars = reinterpret_cast<uint64_t *>(mml + C::MLF);         // full[NS], empty[NS], block
     TileDesc *sdesc = reinterpret_cast<TileDesc *>(bars + 2 * NS + 2);   // [NS]
     int *sflag = reinterpret_cast<int *>(sdesc + NS);                    // [16]
@@ -292,7 +193,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             // partner's partial received: the first CTA of a pair expects its bytes (used only
             // when the pair splits one head; otherwise nothing waits on it)
             mbar_init(smem_addr(&bars[2 * NS + 1]), 1);
-            if (!(blockIdx.x & 1)) mbar_expect_tx(smem_addr(&bars[2 * NS + 1]), a.Mq * (D * 4 + 8));
+            if (!(blockIdx.x & 1)) mbar_expect_tx(smem_addr(&bars[2 * NS + 1]), a.Mq * (D * 4 + 16));
         }
         mbar_fence_init();
     }
@@ -305,76 +206,10 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     }
     // ---- per-sequence tile counts and their prefix sums (T is written by earlier kernels)
     if (!a.early) pdl_wait();
-    int total, chunk, pieces;  // pieces 0: contiguous chunks of the whole tile list
-    int tot_head = 0;          // tiles per (sequence, kv head) in piece mode
-    SeqGeom sg1 = {};          // the sequence's geometry when N == 1
-    if (N == 1) {
-        // one sequence: every thread reads T and cuts the list itself (no scan, no broadcast)
-        const int T = a.T[0];
-        sg1 = seq_geom(T, pa);
-        const int tot0 = sg1.total;
-        tot_head = tot0;
-        total = tot0 * kvH;
-        choose_chunk(total, tot0, true, static_cast<int>(gridDim.x), 1, kvH, a.min_chunk, chunk, pieces);
-        if (tid == 0) {
-            Ts[0] = T;
-            cum[0] = 0;
-            cum[1] = total;
-        }
-        __syncthreads();
-        pdl_trigger();  // the next kernel may be scheduled; it waits for this one to finish
-    } else {
-        for (int n = tid; n < N; n += blockDim.x) {
-            const int T = a.T[n];
-            Ts[n] = T;
-            cum[n + 1] = seq_geom(T, pa).total * kvH;
-        }
-        if (tid == 0) cum[0] = 0;
-        __syncthreads();
-        if (warp == 0) {  // inclusive scan of cum[1..N] in chunks of 32
-            int carry = 0;
-            for (int b = 0; b < N; b += 32) {
-                int v = (b + lane < N) ? cum[b + lane + 1] : 0;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int u = __shfl_up_sync(0xffffffffu, v, o);
-                    if (lane >= o) v += u;
-                }
-                if (b + lane < N) cum[b + lane + 1] = v + carry;
-                carry += __shfl_sync(0xffffffffu, v, 31);
-            }
-        }
-        __syncthreads();
-        pdl_trigger();
-        total = cum[N];
-        if (warp == 0) {
-            // equal tile counts for every (sequence, kv head)?
-            bool same = true;
-            for (int b = 0; b < N; b += 32) {
-                const bool ok = (b + lane >= N) || (cum[b + lane + 1] - cum[b + lane] == cum[1]);
-                same = same && __all_sync(0xffffffffu, ok);
-            }
-            if (lane == 0) {
-                int ch, pc;
-                choose_chunk(total, cum[1] / kvH, same, static_cast<int>(gridDim.x), N, kvH, a.min_chunk, ch, pc);
-                sflag[6] = ch;
-                sflag[7] = pc;
-            }
-        }
-        __syncthreads();
-        chunk = sflag[6];
-        pieces = sflag[7];
-        if (pieces) tot_head = cum[1] / kvH;
-    }
-    int g_begin, g_end, head = 0;
-    if (pieces) {
-        head = blockIdx.x / pieces;
-        g_begin = head * tot_head + (blockIdx.x - head * pieces) * chunk;
-        g_end = min(min(g_begin + chunk, (head + 1) * tot_head), total);
-    } else {
-        g_begin = blockIdx.x * chunk;
-        g_end = min(total, g_begin + chunk);
-    }
+    const ChunkPlan cp = plan_chunks(a, cum, Ts, sflag, tid, warp, lane);
+    const int chunk = cp.chunk, pieces = cp.pieces, head = cp.head;
+    const int g_begin = cp.g_begin, g_end = cp.g_end;
+    const SeqGeom &sg1 = cp.sg1;
     if (g_begin >= g_end) {
         if (a.early) pdl_wait();  // the launch completes only after its predecessor
         return;
@@ -546,7 +381,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     const uint32_t vcol_sel = static_cast<uint32_t>(mi & 1);
 
     float o[D / 16][NQT][4];
-    float m_ref[NQT][2], l_run[NQT][2];
+    // l_run sums the fp32 probabilities (the log-sum-exp); l_bf sums them as rounded to bf16 for
+    // the P V product, so that the output is a true weighted average of V with those weights
+    float m_ref[NQT][2], l_run[NQT][2], l_bf[NQT][2];
     uint32_t qb[D / 16][NQT][2];
 
     int fin_next = P_first;  // next pair to finalize (every consumer warp finalizes each pair once)
@@ -562,6 +399,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         for (int nq = 0; nq < NQT; ++nq) {
             m_ref[nq][0] = m_ref[nq][1] = -INFINITY;
             l_run[nq][0] = l_run[nq][1] = 0.f;
+            l_bf[nq][0] = l_bf[nq][1] = 0.f;
         }
     };
 
@@ -605,11 +443,15 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             for (int nq = 0; nq < NQT; ++nq)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
-                    float l = l_run[nq][e];
+                    float l = l_run[nq][e], lb = l_bf[nq][e];
                     l += __shfl_xor_sync(0xffffffffu, l, 4);
                     l += __shfl_xor_sync(0xffffffffu, l, 8);
                     l += __shfl_xor_sync(0xffffffffu, l, 16);
+                    lb += __shfl_xor_sync(0xffffffffu, lb, 4);
+                    lb += __shfl_xor_sync(0xffffffffu, lb, 8);
+                    lb += __shfl_xor_sync(0xffffffffu, lb, 16);
                     l_run[nq][e] = l;
+                    l_bf[nq][e] = lb;
                 }
 #pragma unroll
             for (int mt = 0; mt < D / 16; ++mt)
@@ -627,15 +469,13 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int q = 8 * nq + 2 * c4 + e;
-                        mml[(warp * C::NQ + q) * 2] = m_ref[nq][e];
-                        mml[(warp * C::NQ + q) * 2 + 1] = l_run[nq][e];
+                        *reinterpret_cast<float4 *>(&mml[(warp * C::NQ + q) * 4]) =
+                            make_float4(m_ref[nq][e], l_bf[nq][e], l_run[nq][e], 0.f);
                     }
             }
         } else {
-            for (int q = lane; q < C::NQ; q += 32) {
-                mml[(warp * C::NQ + q) * 2] = -INFINITY;
-                mml[(warp * C::NQ + q) * 2 + 1] = 0.f;
-            }
+            for (int q = lane; q < C::NQ; q += 32)
+                *reinterpret_cast<float4 *>(&mml[(warp * C::NQ + q) * 4]) = make_float4(-INFINITY, 0.f, 0.f, 0.f);
         }
         named_bar_sync(1, nct);
         const bool abort_now = *reinterpret_cast<volatile int *>(&sflag[1]) != 0;
@@ -649,20 +489,20 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 #pragma unroll
             for (int t2 = 0; t2 < TG; ++t2)
 #pragma unroll
-                for (int k = 0; k < WK; ++k) M = fmaxf(M, mml[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * 2]);
-            float L = 0.f;
+                for (int k = 0; k < WK; ++k) M = fmaxf(M, mml[((t2 * C::GW + rgi * WK + k) * C::NQ + q) * 4]);
+            float L = 0.f, Ll = 0.f;
 #pragma unroll
             for (int t2 = 0; t2 < TG; ++t2)
 #pragma unroll
                 for (int k = 0; k < WK; ++k) {
                     const int w = t2 * C::GW + rgi * WK + k;
-                    const float mk = mml[(w * C::NQ + q) * 2];
-                    const float f = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+                    const float4 ml = *reinterpret_cast<const float4 *>(&mml[(w * C::NQ + q) * 4]);
+                    const float f = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
                     wq[i * (TG * WK) + t2 * WK + k] = f;
-                    L += f * mml[(w * C::NQ + q) * 2 + 1];
+                    L += f * ml.y;
+                    Ll += f * ml.z;
                 }
-            fin[i * 2] = M;
-            fin[i * 2 + 1] = L;
+            *reinterpret_cast<float4 *>(&fin[i * 4]) = make_float4(M, L, Ll, 0.f);
         }
         named_bar_sync(1, nct);
         // four consecutive columns of one row per thread: float4 shared-memory reads (the
@@ -697,7 +537,9 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     const int i = e / D4, c0 = 4 * (e - i * D4);
                     const float4 acc = row_acc(i, c0);
                     st_async_v4(rxo + 4u * static_cast<uint32_t>(i * D + c0), acc, rbar);
-                    if (c0 == 0) st_async_v2(rxml + 8u * static_cast<uint32_t>(i), fin[i * 2], fin[i * 2 + 1], rbar);
+                    if (c0 == 0)
+                        st_async_v4(rxml + 16u * static_cast<uint32_t>(i), *reinterpret_cast<const float4 *>(&fin[i * 4]),
+                                    rbar);
                 }
             } else {
                 // bounded wait for the partner's bytes
@@ -707,18 +549,19 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     const int i = e / D4, c0 = 4 * (e - i * D4);
                     const float4 acc = row_acc(i, c0);
                     const float4 o1 = *reinterpret_cast<const float4 *>(&xo[i * D + c0]);
-                    const float M0 = fin[i * 2], M1 = xml[i * 2];
-                    const float M = fmaxf(M0, M1);
-                    const float w0 = (M0 == -INFINITY) ? 0.f : exp2f(M0 - M);
-                    const float w1 = (M1 == -INFINITY) ? 0.f : exp2f(M1 - M);
-                    const float L = w0 * fin[i * 2 + 1] + w1 * xml[i * 2 + 1];
+                    const float4 f0 = *reinterpret_cast<const float4 *>(&fin[i * 4]);
+                    const float4 f1 = *reinterpret_cast<const float4 *>(&xml[i * 4]);
+                    const float M = fmaxf(f0.x, f1.x);
+                    const float w0 = (f0.x == -INFINITY) ? 0.f : exp2f(f0.x - M);
+                    const float w1 = (f1.x == -INFINITY) ? 0.f : exp2f(f1.x - M);
+                    const float L = w0 * f0.y + w1 * f1.y, Ll = w0 * f0.z + w1 * f1.z;
                     const float inv = 1.f / L;
                     const int j = i / a.g, h = kh * a.g + (i - j * a.g);
                     const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
                     __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + c0]);
                     op[0] = __floats2bfloat162_rn((w0 * acc.x + w1 * o1.x) * inv, (w0 * acc.y + w1 * o1.y) * inv);
                     op[1] = __floats2bfloat162_rn((w0 * acc.z + w1 * o1.z) * inv, (w0 * acc.w + w1 * o1.w) * inv);
-                    if (c0 == 0 && a.lse) a.lse[orow] = (M + __log2f(L)) * 0.69314718055994531f;
+                    if (c0 == 0 && a.lse) a.lse[orow] = (M + __log2f(Ll)) * 0.69314718055994531f;
                 }
                 named_bar_sync(1, nct);
             }
@@ -729,13 +572,13 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             const int i = e / D4, c0 = 4 * (e - i * D4);
             const float4 acc = row_acc(i, c0);  // a warp that saw no key of the row has weight 0
             if (sole) {
-                const float inv = 1.f / fin[i * 2 + 1];
+                const float inv = 1.f / fin[i * 4 + 1];
                 const int j = i / a.g, h = kh * a.g + (i - j * a.g);
                 const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
                 __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + c0]);
                 op[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
                 op[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-                if (c0 == 0 && a.lse) a.lse[orow] = (fin[i * 2] + __log2f(fin[i * 2 + 1])) * 0.69314718055994531f;
+                if (c0 == 0 && a.lse) a.lse[orow] = (fin[i * 4] + __log2f(fin[i * 4 + 2])) * 0.69314718055994531f;
             } else {
                 if (kDebug && static_cast<int>(blockIdx.x) + p >= a.dbg_part_slots) {
                     atomicOr(a.err, RIPE_DEVERR_BOUNDS);
@@ -743,10 +586,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 }
                 const size_t prow = (static_cast<size_t>(blockIdx.x) + p) * C::ROWS + i;
                 *reinterpret_cast<float4 *>(&a.part_o[prow * D + c0]) = acc;
-                if (c0 == 0) {
-                    a.part_ml[prow * 2] = fin[i * 2];
-                    a.part_ml[prow * 2 + 1] = fin[i * 2 + 1];
-                }
+                if (c0 == 0) *reinterpret_cast<float4 *>(&a.part_ml[prow * 4]) = *reinterpret_cast<const float4 *>(&fin[i * 4]);
             }
         }
         named_bar_sync(1, nct);  // partials written; the merge buffer is free again
@@ -770,11 +610,11 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         const int nparts = parts_of(p, c_first);
         float *pw = reinterpret_cast<float *>(stages);  // [nparts][ROWS] m, then weights
         float *pl = pw + nparts * C::ROWS;              // [nparts][ROWS] l
-        float *rowML = fin;                             // [ROWS][2] final M, L
+        float *rowML = fin;                             // [ROWS][4] final M, L_out, L_lse
         for (int e = tid; e < nparts * a.Mq; e += nct) {
             const int c = e / a.Mq, i = e - (e / a.Mq) * a.Mq;
             const size_t prow = (static_cast<size_t>(c_first + c) + p) * C::ROWS + i;
-            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(&a.part_ml[prow * 2]));
+            const float2 ml = __ldcg(reinterpret_cast<const float2 *>(&a.part_ml[prow * 4]));
             pw[c * C::ROWS + i] = ml.x;
             pl[c * C::ROWS + i] = ml.y;
         }
@@ -782,15 +622,18 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         for (int i = tid; i < a.Mq; i += nct) {
             float M = -INFINITY;
             for (int c = 0; c < nparts; ++c) M = fmaxf(M, pw[c * C::ROWS + i]);
-            float L = 0.f;
+            float L = 0.f, Ll = 0.f;
             for (int c = 0; c < nparts; ++c) {
                 const float mk = pw[c * C::ROWS + i];
                 const float w = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
                 pw[c * C::ROWS + i] = w;
                 L += w * pl[c * C::ROWS + i];
+                const size_t prow = (static_cast<size_t>(c_first + c) + p) * C::ROWS + i;
+                Ll += w * __ldcg(&a.part_ml[prow * 4 + 2]);
             }
-            rowML[i * 2] = M;
-            rowML[i * 2 + 1] = L;
+            rowML[i * 4] = M;
+            rowML[i * 4 + 1] = L;
+            rowML[i * 4 + 2] = Ll;
         }
         named_bar_sync(1, nct);
         for (int e = tid; e < a.Mq * (D / 4); e += nct) {
@@ -803,14 +646,14 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     &a.part_o[((static_cast<size_t>(c_first + c) + p) * C::ROWS + i) * D + 4 * c4x]));
                 acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
             }
-            const float invL = 1.f / rowML[i * 2 + 1];
+            const float invL = 1.f / rowML[i * 4 + 1];
             const int j = i / a.g, h = kh * a.g + (i - j * a.g);
             const size_t orow = (static_cast<size_t>(n) * a.qB + j) * a.Hq + h;
             __nv_bfloat162 *op = reinterpret_cast<__nv_bfloat162 *>(&a.out[orow * D + 4 * c4x]);
             op[0] = __floats2bfloat162_rn(acc.x * invL, acc.y * invL);
             op[1] = __floats2bfloat162_rn(acc.z * invL, acc.w * invL);
             if (c4x == 0 && a.lse)
-                a.lse[orow] = (rowML[i * 2] + __log2f(rowML[i * 2 + 1])) * 0.69314718055994531f;
+                a.lse[orow] = (rowML[i * 4] + __log2f(rowML[i * 4 + 2])) * 0.69314718055994531f;
         }
         if (tid == 0) a.counters[p] = 0;
         named_bar_sync(1, nct);
@@ -895,6 +738,8 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
             for (int nq = 0; nq < NQT; ++nq) {
                 l_run[nq][0] *= alpha[nq][0];
                 l_run[nq][1] *= alpha[nq][1];
+                l_bf[nq][0] *= alpha[nq][0];
+                l_bf[nq][1] *= alpha[nq][1];
 #pragma unroll
                 for (int mt = 0; mt < D / 16; ++mt) {
                     o[mt][nq][0] *= alpha[nq][0]; o[mt][nq][1] *= alpha[nq][1];
@@ -917,10 +762,12 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 const float p3 = (r1 == -INFINITY) ? 0.f : exp2f(x[sb][nq][3] - r1);
                 const __nv_bfloat162 lo = __floats2bfloat162_rn(p0, p1);
                 const __nv_bfloat162 hi = __floats2bfloat162_rn(p2, p3);
-                // the normaliser sums the fp32 probabilities (the lse stays fp32-accurate);
-                // only the P V product sees them rounded to bf16
+                // two normalisers: the rounded probabilities the P V product sees (the output is
+                // their weighted average of V) and the fp32 ones (the lse stays fp32-accurate)
                 l_run[nq][0] += p0 + p2;
                 l_run[nq][1] += p1 + p3;
+                l_bf[nq][0] += __low2float(lo) + __low2float(hi);
+                l_bf[nq][1] += __high2float(lo) + __high2float(hi);
                 pb[nq][0] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&lo));
                 pb[nq][1] = movmatrix_t(*reinterpret_cast<const uint32_t *>(&hi));
             }
@@ -998,12 +845,6 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 // allocation or call ever lowers it below what a live cache of a larger batch needs.
 template <class C>
 constexpr int kSmemMax = smem_bytes_for<C>(kMaxBatch);
-
-// Where a verify launch reads from: the four tensor maps, the device and its SM count.
-struct LaunchTarget {
-    const CUtensorMap *tmKd, *tmVd, *tmKw, *tmVw;
-    int device, num_sms, N;
-};
 
 template <int D, int NQT, int WR, int WK, int TG>
 struct Inst {
@@ -1099,6 +940,7 @@ int ensure_verify_attributes(int device) {
     cudaError_t e = set_all_max<RIPE_QCFG_LIST(64)>();
     if (e == cudaSuccess) e = set_all_max<RIPE_QCFG_LIST(96)>();
     if (e == cudaSuccess) e = set_all_max<RIPE_QCFG_LIST(128)>();
+    if (e == cudaSuccess) e = set_verify_tc_attributes();
     if (e != cudaSuccess) {
         cudaGetLastError();
         return RIPE_ECUDA;
@@ -1117,7 +959,20 @@ static cudaError_t launch_d(int qc, const LaunchTarget &t, int grid, const Verif
     }
 }
 
+// The consumer for 9..64 query rows per kv head: the tcgen05 kernel (ripe_verify_tc.cu), unless the
+// environment variable RIPE_VERIFY_CONSUMER is "mma" (the mma.sync consumer of this file; for A/B
+// timing).  Launches that write the draft block (fused append, draft steps) always use this file's
+// kernel.
+static bool tc_consumer() {
+    static const bool use = [] {
+        const char *e = std::getenv("RIPE_VERIFY_CONSUMER");
+        return !(e && std::strcmp(e, "mma") == 0);
+    }();
+    return use;
+}
+
 static cudaError_t launch_any(int d, int qc, const LaunchTarget &t, int grid, const VerifyArgs &a, cudaStream_t s) {
+    if (qc >= 1 && a.blk_k == nullptr && tc_consumer()) return launch_verify_tc(d, t, grid, a, s);
     switch (d) {
         case 64: return launch_d<RIPE_QCFG_LIST(64)>(qc, t, grid, a, s);
         case 96: return launch_d<RIPE_QCFG_LIST(96)>(qc, t, grid, a, s);

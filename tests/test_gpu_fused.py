@@ -1,12 +1,16 @@
-"""ripe_append_verify == ripe_append_block + ripe_verify_attn, bit for bit: the outputs of every
-call and the cache state after each commit, over several decode steps with ragged accepted
-lengths (ring wrap-around, eviction, all three layouts); and ripe_append_verify against the CPU
-oracle directly."""
+"""ripe_append_verify == ripe_append_block + ripe_verify_attn: the cache state after each commit bit
+for bit, and the outputs of every call bit for bit when both calls run the same consumer (up to 8
+query rows per kv head, or every size with RIPE_VERIFY_CONSUMER=mma; otherwise the separate call runs
+the tcgen05 consumer and the two outputs agree within the parity tolerance), over several decode
+steps with ragged accepted lengths (ring wrap-around, eviction, all three layouts); and
+ripe_append_verify against the CPU oracle directly."""
+import os
+
 import numpy as np
 import pytest
 import torch
 
-from harness import Case, check_close, check_lse, dev_to_bits
+from harness import Case, assert_same_result, check_close, check_lse, dev_to_bits
 from self_speculative_decode_b200.ripe import RipeCache
 from self_speculative_decode_b200.synth import PlaneSource, acceptance_draws
 
@@ -19,6 +23,9 @@ pytestmark = pytest.mark.gpu
 def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, T0, cuda_device):
     """T0 = 60 (full cache) and 188 (deepest only) put the block's rows across a 64-row tile edge."""
     N, L, kvH, R, steps = 3, 2, 3, 4, 6
+    # the fused launch always runs the mma.sync consumer; a separate verify with more than 8 query rows
+    # per kv head runs the tcgen05 one unless RIPE_VERIFY_CONSUMER=mma
+    same_consumer = B * g <= 8 or os.environ.get("RIPE_VERIFY_CONSUMER") == "mma"
     max_T = T0 + B * (steps + 1)
     src = PlaneSource(N, kvH, d, R, T0, 0.88, 31, backend="torch", device=cuda_device)
     caches = [RipeCache(N, L, kvH * g, kvH, d, R, W, max_T, B) for _ in range(2)]
@@ -38,7 +45,10 @@ def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, T0, cuda_devic
                 caches[0].append_block(layer, r, kb, vb)
                 a = caches[0].verify_attn(layer, r, q)
                 b = caches[1].append_verify(layer, r, kb, vb, q)
-                assert torch.equal(a, b), (step, r, layer)
+                if same_consumer:
+                    assert torch.equal(a, b), (step, r, layer)
+                else:
+                    assert_same_result(a, b, f"step {step} loop {r} layer {layer}")
         for c in caches:
             c.commit(acc[step])
         for n in range(N):
