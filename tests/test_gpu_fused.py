@@ -1,7 +1,8 @@
 """ripe_append_verify == ripe_append_block + ripe_verify_attn: the cache state after each commit bit
-for bit, and the outputs of every call bit for bit when both calls run the same consumer (up to 8
-query rows per kv head, or every size with RIPE_VERIFY_CONSUMER=mma; otherwise the separate call runs
-the tcgen05 consumer and the two outputs agree within the parity tolerance), over several decode
+for bit, and the outputs of every call bit for bit when both calls run the same consumer (the fused
+call always runs the mma.sync one; at these sizes so does the separate call, unless
+RIPE_VERIFY_CONSUMER=tc puts the tcgen05 one on 9..64 query rows per kv head, and then the two
+outputs agree within the parity tolerance), over several decode
 steps with ragged accepted lengths (ring wrap-around, eviction, all three layouts); and
 ripe_append_verify against the CPU oracle directly."""
 import os
@@ -23,9 +24,9 @@ pytestmark = pytest.mark.gpu
 def test_fused_append_verify_is_bitwise_the_two_calls(W, B, g, d, T0, cuda_device):
     """T0 = 60 (full cache) and 188 (deepest only) put the block's rows across a 64-row tile edge."""
     N, L, kvH, R, steps = 3, 2, 3, 4, 6
-    # the fused launch always runs the mma.sync consumer; a separate verify with more than 8 query rows
-    # per kv head runs the tcgen05 one unless RIPE_VERIFY_CONSUMER=mma
-    same_consumer = B * g <= 8 or os.environ.get("RIPE_VERIFY_CONSUMER") == "mma"
+    # the fused launch always runs the mma.sync consumer; a separate verify of these short pairs
+    # runs it too unless RIPE_VERIFY_CONSUMER=tc puts the tcgen05 one on 9..64 query rows
+    same_consumer = B * g <= 8 or os.environ.get("RIPE_VERIFY_CONSUMER") != "tc"
     max_T = T0 + B * (steps + 1)
     src = PlaneSource(N, kvH, d, R, T0, 0.88, 31, backend="torch", device=cuda_device)
     caches = [RipeCache(N, L, kvH * g, kvH, d, R, W, max_T, B) for _ in range(2)]
