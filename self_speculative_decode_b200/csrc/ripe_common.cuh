@@ -256,6 +256,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
     }
 }
 
+// ---- register reallocation between warpgroups (all threads of a warpgroup execute the same one)
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---- thread-block clusters (a pair of CTAs exchanging partial results in shared memory)
 // every thread of every CTA of the cluster: arrive (release) and wait (acquire)
 __device__ __forceinline__ void cluster_sync_all() {

@@ -17,6 +17,8 @@
 //   * One producer thread streams 64-key K/V tiles with 3-D TMA loads (64-byte swizzle, no
 //     multicast) into a shared-memory ring of NS stages guarded by mbarriers, and writes a
 //     small descriptor of each tile (sequence, kv head, kind, first key, count) beside it.
+//     Its warp heads a warpgroup of its own that gives registers up (setmaxnreg) to the two
+//     consumer warpgroups, so that their fragments of Q, O and S fit without spilling.
 //   * Consumer warps work on the transposed problem S^T = K Q^T (keys on the MMA's M side,
 //     the B x group query rows on its N side, so an 8-row block is not padded to 16), with
 //     mma.sync m16n8k16 bf16 -> fp32.  P^T is moved into the B-operand layout of
@@ -49,7 +51,19 @@ struct VCfg {
     static constexpr int ROWS = NQ * WR;           // query rows per (sequence, kv head)
     static constexpr int GW = WR * WK;             // warps per tile group
     static constexpr int NCW = GW * TG;            // consumer warps
-    static constexpr int THREADS = (NCW + 1) * 32; // + the producer warp
+    // + one warpgroup: the producer warp, the copy warp of the fused form and two idle warps.  The
+    // consumer warpgroups take the registers that the producer warpgroup gives up (setmaxnreg):
+    // launched at LAUNCH_REGS per thread, they run at REG_CONSUMER, the producer group at
+    // REG_PRODUCER, and the split adds up to no more than the launch's registers.
+    static constexpr int THREADS = (NCW + 4) * 32;
+    static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8 > 255 ? 248 : (65536 / THREADS) / 8 * 8;
+    static constexpr int REG_PRODUCER = 72;
+    static constexpr int REG_CONSUMER =
+        ((LAUNCH_REGS * (NCW + 4) - 4 * REG_PRODUCER) / NCW) / 8 * 8 > 248
+            ? 248
+            : ((LAUNCH_REGS * (NCW + 4) - 4 * REG_PRODUCER) / NCW) / 8 * 8;
+    static_assert(NCW % 4 == 0, "consumer warps form whole warpgroups");
+    static_assert(NCW * REG_CONSUMER + 4 * REG_PRODUCER <= (NCW + 4) * LAUNCH_REGS, "register split");
     static constexpr int SB = 4 / WK;              // 16-key sub-blocks per warp per tile
     static constexpr int NBOX = D / kBoxCols;
     static constexpr int STAGE_BYTES = 2 * NBOX * kBoxBytes;
@@ -145,7 +159,7 @@ __device__ __noinline__ int first_written_tile(SeqGeom sg, int lt, int n, int kh
 
 // FUSED adds one warp after the producer that writes the draft block's rows into the ring.
 template <int D, int NQT, int WR, int WK, int TG, bool FUSED>
-__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS + (FUSED ? 32 : 0), 1)
+__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS, 1)
 ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_constant__ CUtensorMap tmVd,
                    const __grid_constant__ CUtensorMap tmKw, const __grid_constant__ CUtensorMap tmVw,
                    const __grid_constant__ VerifyArgs a) {
@@ -226,19 +240,22 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     // FUSED (ripe_append_verify, draft steps): a copy warp writes the block rows into the ring; a
     // separate instantiation so that plain verification carries none of that code
     constexpr bool fused = FUSED;
-    if constexpr (fused) {
-        if (warp == C::NCW + 1) {
-            // the copy warp: write the draft block's rows that this CTA's tiles read into the
-            // ring, fence them for the TMA (async proxy), release the producer
-            if (a.early) pdl_wait();  // the caller's block rows and the ring slots they replace
-            fused_block_copy<D>(a, cum, Ts, g_begin, g_end, lane, 32);
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&bars[2 * NS]));
-            return;
+    if (warp >= C::NCW) {
+        // the producer warpgroup hands registers to the consumers
+        setmaxnreg_dec<C::REG_PRODUCER>();
+        if constexpr (fused) {
+            if (warp == C::NCW + 1) {
+                // the copy warp: write the draft block's rows that this CTA's tiles read into the
+                // ring, fence them for the TMA (async proxy), release the producer
+                if (a.early) pdl_wait();  // the caller's block rows and the ring slots they replace
+                fused_block_copy<D>(a, cum, Ts, g_begin, g_end, lane, 32);
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&bars[2 * NS]));
+                return;
+            }
         }
-    }
-    if (warp == C::NCW) {
+        if (warp != C::NCW) return;
         // ================================================================ producer (one thread)
         if (lane != 0 && a.early) {
             // the other lanes bring the first pair's query rows into L2 while the previous launch
@@ -351,6 +368,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         }
         return;  // the producer warp takes part in no consumer barrier (id 1)
     }
+    setmaxnreg_inc<C::REG_CONSUMER>();
 
 
     // ==================================================================== consumers
@@ -852,8 +870,22 @@ struct Inst {
     static_assert(kSmemMax<C> <= kSmemLimit, "the largest batch's shared memory must fit a CTA");
     static constexpr auto kernel = ripe_verify_kernel<D, NQT, WR, WK, TG, false>;
     static constexpr auto kernel_fused = ripe_verify_kernel<D, NQT, WR, WK, TG, true>;
+    // The register split assumes the kernels are launched at LAUNCH_REGS per thread; with fewer, the
+    // consumers' setmaxnreg.inc could never be satisfied: refuse the kernels instead.
+    static cudaError_t check_registers() {
+        for (auto k : {kernel, kernel_fused}) {
+            cudaFuncAttributes fa;
+            const cudaError_t e = cudaFuncGetAttributes(&fa, k);
+            if (e != cudaSuccess) return e;
+            if (fa.numRegs * C::THREADS < C::NCW * 32 * C::REG_CONSUMER + 4 * 32 * C::REG_PRODUCER)
+                return cudaErrorInvalidConfiguration;
+        }
+        return cudaSuccess;
+    }
     static cudaError_t set_attr_max() {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax<C>);
+        cudaError_t e = check_registers();
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax<C>);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(kernel_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax<C>);
         return e;
@@ -870,7 +902,7 @@ struct Inst {
         std::lock_guard<std::mutex> lock(mu);
         Entry &e = cache[device][f];
         if (e.smem != smem) {
-            const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::THREADS + 32 * f), smem, 2,
+            const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::THREADS), smem, 2,
                                               num_sms & ~1);
             e.grid = 2 * n;
             e.smem = smem;
@@ -881,7 +913,7 @@ struct Inst {
         if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
         const bool fused = args.blk_k != nullptr;
         auto kern = fused ? kernel_fused : kernel;
-        const dim3 block(C::THREADS + (fused ? 32 : 0));
+        const dim3 block(C::THREADS);
         const int smem = smem_bytes_for<C>(t.N);
         VerifyArgs a = args;
         a.xpair = 0;
