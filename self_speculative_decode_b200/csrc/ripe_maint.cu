@@ -28,8 +28,11 @@ __global__ void ripe_append_kernel(uint4 *__restrict__ Kw, uint4 *__restrict__ V
                                    const uint4 *__restrict__ k, const uint4 *__restrict__ v,
                                    const int32_t *__restrict__ T, uint32_t *err, int N, int B, int kvH,
                                    int d8, int R, int S, int layer, int r, int max_T) {
-    pdl_wait();
+    // The next launch may start at once: a verify launch reads nothing this kernel writes before
+    // its own wait, which returns only after this kernel (and so its predecessor) has completed.
+    // Its CTAs then take the SMs that the previous verify launch leaves, while this one waits.
     pdl_trigger();
+    pdl_wait();
     const size_t total = static_cast<size_t>(N) * B * kvH * d8;
     for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
          idx += static_cast<size_t>(gridDim.x) * blockDim.x) {

@@ -17,8 +17,9 @@
 //   * One producer thread streams 64-key K/V tiles with 3-D TMA loads (64-byte swizzle, no
 //     multicast) into a shared-memory ring of NS stages guarded by mbarriers, and writes a
 //     small descriptor of each tile (sequence, kv head, kind, first key, count) beside it.
-//     Its warp heads a warpgroup of its own that gives registers up (setmaxnreg) to the two
-//     consumer warpgroups, so that their fragments of Q, O and S fit without spilling.
+//     For two query tiles per warp its warp heads a warpgroup of its own that gives registers
+//     up (setmaxnreg) to the two consumer warpgroups, so that their fragments of Q, O and S fit
+//     without spilling.
 //   * Consumer warps work on the transposed problem S^T = K Q^T (keys on the MMA's M side,
 //     the B x group query rows on its N side, so an 8-row block is not padded to 16), with
 //     mma.sync m16n8k16 bf16 -> fp32.  P^T is moved into the B-operand layout of
@@ -51,11 +52,16 @@ struct VCfg {
     static constexpr int ROWS = NQ * WR;           // query rows per (sequence, kv head)
     static constexpr int GW = WR * WK;             // warps per tile group
     static constexpr int NCW = GW * TG;            // consumer warps
-    // + one warpgroup: the producer warp, the copy warp of the fused form and two idle warps.  The
-    // consumer warpgroups take the registers that the producer warpgroup gives up (setmaxnreg):
-    // launched at LAUNCH_REGS per thread, they run at REG_CONSUMER, the producer group at
-    // REG_PRODUCER, and the split adds up to no more than the launch's registers.
-    static constexpr int THREADS = (NCW + 4) * 32;
+    // Threads: the consumers, the producer warp and (fused form) the copy warp.  With two query
+    // tiles per warp (SPLIT), whose Q, O and S fragments do not fit the 168 registers that three
+    // warps per sub-partition leave, the producer and copy warps are padded to a warpgroup that
+    // gives registers up (setmaxnreg) to the consumer warpgroups: launched at LAUNCH_REGS per
+    // thread, they run at REG_CONSUMER, the producer group at REG_PRODUCER, and the split adds up
+    // to no more than the launch's registers.  Without it a CTA keeps enough registers free for a
+    // small kernel (the append) to share the SM.
+    static constexpr bool SPLIT = NQT >= 2;
+    static constexpr int THREADS = SPLIT ? (NCW + 4) * 32 : (NCW + 1) * 32;
+    static constexpr int threads(bool fused) { return THREADS + (fused && !SPLIT ? 32 : 0); }
     static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8 > 255 ? 248 : (65536 / THREADS) / 8 * 8;
     static constexpr int REG_PRODUCER = 72;
     static constexpr int REG_CONSUMER =
@@ -159,7 +165,7 @@ __device__ __noinline__ int first_written_tile(SeqGeom sg, int lt, int n, int kh
 
 // FUSED adds one warp after the producer that writes the draft block's rows into the ring.
 template <int D, int NQT, int WR, int WK, int TG, bool FUSED>
-__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::THREADS, 1)
+__global__ void __launch_bounds__(VCfg<D, NQT, WR, WK, TG>::threads(FUSED), 1)
 ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_constant__ CUtensorMap tmVd,
                    const __grid_constant__ CUtensorMap tmKw, const __grid_constant__ CUtensorMap tmVw,
                    const __grid_constant__ VerifyArgs a) {
@@ -242,7 +248,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
     constexpr bool fused = FUSED;
     if (warp >= C::NCW) {
         // the producer warpgroup hands registers to the consumers
-        setmaxnreg_dec<C::REG_PRODUCER>();
+        if constexpr (C::SPLIT) setmaxnreg_dec<C::REG_PRODUCER>();
         if constexpr (fused) {
             if (warp == C::NCW + 1) {
                 // the copy warp: write the draft block's rows that this CTA's tiles read into the
@@ -368,7 +374,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         }
         return;  // the producer warp takes part in no consumer barrier (id 1)
     }
-    setmaxnreg_inc<C::REG_CONSUMER>();
+    if constexpr (C::SPLIT) setmaxnreg_inc<C::REG_CONSUMER>();
 
 
     // ==================================================================== consumers
@@ -873,12 +879,14 @@ struct Inst {
     // The register split assumes the kernels are launched at LAUNCH_REGS per thread; with fewer, the
     // consumers' setmaxnreg.inc could never be satisfied: refuse the kernels instead.
     static cudaError_t check_registers() {
-        for (auto k : {kernel, kernel_fused}) {
-            cudaFuncAttributes fa;
-            const cudaError_t e = cudaFuncGetAttributes(&fa, k);
-            if (e != cudaSuccess) return e;
-            if (fa.numRegs * C::THREADS < C::NCW * 32 * C::REG_CONSUMER + 4 * 32 * C::REG_PRODUCER)
-                return cudaErrorInvalidConfiguration;
+        if constexpr (C::SPLIT) {
+            for (auto k : {kernel, kernel_fused}) {
+                cudaFuncAttributes fa;
+                const cudaError_t e = cudaFuncGetAttributes(&fa, k);
+                if (e != cudaSuccess) return e;
+                if (fa.numRegs * C::THREADS < C::NCW * 32 * C::REG_CONSUMER + 4 * 32 * C::REG_PRODUCER)
+                    return cudaErrorInvalidConfiguration;
+            }
         }
         return cudaSuccess;
     }
@@ -902,7 +910,7 @@ struct Inst {
         std::lock_guard<std::mutex> lock(mu);
         Entry &e = cache[device][f];
         if (e.smem != smem) {
-            const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::THREADS), smem, 2,
+            const int n = max_active_clusters(fused ? kernel_fused : kernel, dim3(C::threads(fused)), smem, 2,
                                               num_sms & ~1);
             e.grid = 2 * n;
             e.smem = smem;
@@ -913,7 +921,7 @@ struct Inst {
         if (grid > C::MAX_PARTS) grid = C::MAX_PARTS;
         const bool fused = args.blk_k != nullptr;
         auto kern = fused ? kernel_fused : kernel;
-        const dim3 block(C::THREADS);
+        const dim3 block(C::threads(fused));
         const int smem = smem_bytes_for<C>(t.N);
         VerifyArgs a = args;
         a.xpair = 0;
