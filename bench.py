@@ -49,6 +49,9 @@ CONFIGS = {
     "long_gqa": dict(N=8, L=4, Hq=32, kvH=8, d=128, R=32, T=32768, W=64, B=8, rho=0.85,
                      workload="Long-context GQA: 4 recurrent layers, 32 q / 8 kv heads x 128, R=32, "
                               "T=32768, W=64, B=8, batch 8, rho 0.85"),
+    "gqa64": dict(N=8, L=4, Hq=64, kvH=8, d=128, R=32, T=32768, W=64, B=8, rho=0.85,
+                  workload="Long-context GQA, 64 query rows per kv head: 4 recurrent layers, 64 q / 8 kv "
+                           "heads x 128, R=32, T=32768, W=64, B=8, batch 8, rho 0.85"),
     "huginn": dict(N=1, L=4, Hq=55, kvH=55, d=96, R=32, T=1024, W=64, B=8, rho=0.88,
                    workload="Huginn-shaped verify: 4 recurrent layers, 55 MHA heads x 96, R=32, "
                             "T=1024, W=64, B=8, batch 1, rho 0.88"),
@@ -135,9 +138,8 @@ def sources_digest():
     return h.hexdigest()
 
 
-def captured_traffic(config, T=None):
-    """DRAM bytes per verify launch from the committed ncu summary, if it matches these sources
-    and (when the summary records it) was taken at the committed length T the bench used."""
+def captured_traffic(config):
+    """DRAM bytes per verify launch from the committed ncu summary, if it matches these sources."""
     path = os.path.join(ROOT, "profiles", "ripe_verify_traffic.txt")
     try:
         kv = {}
@@ -156,12 +158,34 @@ def captured_traffic(config, T=None):
         return None
 
 
-def traffic_at(config, T0):
-    """Captured DRAM bytes per launch for this config if the capture was taken at committed length T0."""
+def traffic_for(config, alg_bytes):
+    """DRAM bytes per timed verify launch: the captured launch's bytes, scaled by algorithmic bytes
+    from the captured launch (the committed prefix length) to the timed ones (a few blocks longer;
+    a launch's traffic grows with the key rows it reads)."""
     t = captured_traffic(config)
-    if t and (t["T"] is None or t["T"] == T0):
-        return t["bytes_per_launch"]
-    return None
+    if not t:
+        return None
+    if t["algorithmic_bytes"]:
+        return t["bytes_per_launch"] * alg_bytes / t["algorithmic_bytes"]
+    return t["bytes_per_launch"]
+
+
+def traffic_basis(config):
+    t = captured_traffic(config)
+    if not t:
+        return "no ncu capture of these sources for this config"
+    return (f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at T = {t['T']} (cold L2), "
+            "scaled by algorithmic bytes to the timed launches")
+
+
+def verify_kernel_name(cfg):
+    """The verify kernel the library picks for this workload's launches (its default dispatch):
+    the tcgen05 consumer for head_dim 128 with 57..64 query rows per kv head on long pairs."""
+    rows = cfg["B"] * cfg["Hq"] // cfg["kvH"]
+    tiles_per_cta = cfg["N"] * cfg["kvH"] * (cfg["T"] // 64) / 148
+    consumer = os.environ.get("RIPE_VERIFY_CONSUMER")
+    tc = consumer == "tc" and rows > 8 or (consumer != "mma" and cfg["d"] == 128 and rows >= 57 and tiles_per_cta >= 128)
+    return "ripe_verify_tc_kernel" if tc else "ripe_verify_kernel"
 
 
 def wave_loops(cfg):
@@ -725,7 +749,7 @@ def huginn_extra(args, device, peak, l2):
            "layouts": {k: layout_summary(r, peak) for k, r in res.items()},
            "roofline": {"achieved": v["warm"]["gbs"], "frac": v["warm"]["frac"], "launch_us": v["warm"]["us_per_launch"],
                         "bytes_per_launch": v["warm"]["bytes_per_launch"],
-                        "traffic": traffic_at("huginn", v["T"][0])},
+                        "traffic": traffic_for("huginn", v["warm"]["bytes_per_launch"])},
            "roofline_cold": {"achieved": v["cold"]["gbs"], "frac": v["cold"]["frac"],
                              "launch_us": v["cold"]["us_per_launch"]},
            "l2": l2_note(v["warm"]["bytes_per_launch"], step_distinct_bytes(cfg, v["T"][0], cfg["W"], cfg["L"]), l2),
@@ -1136,7 +1160,7 @@ def main():
     v = m["verify"]
     value = job_throughput(m["bytes_per_step"] * args.steps, m["ms_per_step"] * args.steps, world)
     T_bench = v["T"]
-    traffic_val = traffic_at(args.config, T_bench[0])
+    traffic_val = traffic_for(args.config, v["warm"]["bytes_per_launch"])
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
@@ -1155,8 +1179,9 @@ def main():
         "layouts": {k: dict(layout_summary(r, peak), layers=layout_cfg[k]["L"]) for k, r in results.items()},
         "roofline": {"bound": "hbm", "achieved": v["warm"]["gbs"], "peak": peak, "unit": "GB/s",
                      "frac": v["warm"]["frac"], "traffic": traffic_val, "peak_kind": peak_kind,
-                     "kernel": "ripe_verify_kernel", "launch_us": v["warm"]["us_per_launch"],
+                     "kernel": verify_kernel_name(cfg), "launch_us": v["warm"]["us_per_launch"],
                      "bytes_per_launch": v["warm"]["bytes_per_launch"], "T": T_bench,
+                     "traffic_basis": traffic_basis(args.config),
                      "note": "R*L verify launches back to back as in the step"},
         "roofline_cold": {"achieved": v["cold"]["gbs"], "frac": v["cold"]["frac"],
                           "launch_us": v["cold"]["us_per_launch"], "note": "L2 flushed before each launch"},
