@@ -84,6 +84,10 @@ struct VCfg {
     static constexpr int AVAIL = kSmemLimit - MISC - 4 * (MERGE_FLOATS + MLF) - 4 * (2 * kMaxBatch + 2);
     static constexpr int CAP = (D == 128 && TG == 1) ? RIPE_MAX_STAGES_WIDE : RIPE_MAX_STAGES;
     static constexpr int NS_RAW = AVAIL / STAGE_BYTES > CAP ? CAP : AVAIL / STAGE_BYTES;
+    // A multiple of TG: a stage's previous tile then belongs to the same tile group, whose wait on
+    // it has completed.  With a stage shared by both groups, a group could wait on a tile whose
+    // stage still carries the other group's older tile in flight; the parity test would pass one
+    // phase early and the group would read that tile's data and descriptor.
     static constexpr int NS = NS_RAW - NS_RAW % TG;
     static_assert(NS >= 2, "not enough shared memory for the pipeline");
     static constexpr int SMEM_FIXED = MISC + NS * STAGE_BYTES + 4 * (MERGE_FLOATS + MLF);
