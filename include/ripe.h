@@ -156,7 +156,12 @@ int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, c
  * Work: split-KV over the deepest-plane region and the window ring in one persistent
  * launch; partial results are merged in the same launch, through the shared memory of a
  * 2-CTA cluster when two CTAs share a (sequence, kv head), else through per-call scratch
- * owned by the cache.
+ * owned by the cache.  The contractions run on mma.sync tensor-core tiles, or on the tcgen05
+ * tensor cores (accumulators in tensor memory) for head_dim 128 with 57..64 query rows per kv
+ * head when the host copy of the lengths shows at least 128 key tiles per CTA.  The
+ * environment variable RIPE_VERIFY_CONSUMER = "tc" or "mma", read once per process, puts one
+ * of the two on every launch with 9..64 query rows; the results agree within the bf16 output
+ * rounding, not bit for bit.
  */
 int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out, float *lse,
                      float scale, void *stream);
