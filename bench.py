@@ -67,7 +67,7 @@ CONFIGS = {
 }
 SWEEP_W = (0, 8, 64, 256, 4096)
 SWEEP_B = (4, 8, 16)
-EXTRAS = ("huginn", "sweep", "streaming", "fixed_memory")
+EXTRAS = ("huginn", "gqa64", "sweep", "streaming", "fixed_memory")
 FIXED_MEMORY_GB = 20.0
 
 
@@ -766,6 +766,26 @@ def huginn_extra(args, device, peak, l2):
     return out
 
 
+def gqa64_extra(args, device, peak, l2):
+    """Long-context GQA with 64 query rows per kv head (8 q heads per kv head): the launches the
+    library sends to its tcgen05 consumer.  RIPE layout: the step, each verify launch warm and
+    cold against the roofline, and the wavefront call."""
+    cfg = CONFIGS["gqa64"]
+    sub = argparse.Namespace(**vars(args))
+    m = bench_layout(cfg, "ripe", sub, args.seed, device, False, peak, want_extras=False)
+    v = m["verify"]
+    return {"workload": cfg["workload"], "kernel": verify_kernel_name(cfg),
+            "layouts": {"ripe": layout_summary(m, peak)},
+            "roofline": {"achieved": v["warm"]["gbs"], "frac": v["warm"]["frac"],
+                         "launch_us": v["warm"]["us_per_launch"], "bytes_per_launch": v["warm"]["bytes_per_launch"],
+                         "traffic": traffic_for("gqa64", v["warm"]["bytes_per_launch"]),
+                         "traffic_basis": traffic_basis("gqa64")},
+            "roofline_cold": {"achieved": v["cold"]["gbs"], "frac": v["cold"]["frac"],
+                              "launch_us": v["cold"]["us_per_launch"]},
+            "l2": l2_note(v["warm"]["bytes_per_launch"], step_distinct_bytes(cfg, v["T"][0], cfg["W"], cfg["L"]), l2),
+            "wavefront": {"loops": m["wave"]["loops"], "ripe_us": m["wave"]["us_per_call"], "ripe_gbs": m["wave"]["gbs"]}}
+
+
 def sweep_extra(args, device, peak):
     """All 15 (W, B) points of the window/block sweep on one layer: per-launch verify latency
     (warm, and cold with L2 flushed), the step, and the wavefront call; the full cache's step
@@ -1148,6 +1168,8 @@ def main():
     for name in extras:
         if name == "huginn" and args.config != "huginn":
             extra_out["huginn"] = huginn_extra(args, device, peak, l2)
+        elif name == "gqa64" and args.config != "gqa64":
+            extra_out["gqa64"] = gqa64_extra(args, device, peak, l2)
         elif name == "sweep":
             extra_out["sweep"] = sweep_extra(args, device, peak)
         elif name == "streaming":
