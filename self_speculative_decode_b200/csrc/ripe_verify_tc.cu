@@ -379,10 +379,10 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
             constexpr uint32_t idS = idesc_bf16_m64(64, false);  // S = Q K^T: B (K tile) K-major
             constexpr uint32_t idO = idesc_bf16_m64(D, true);    // O += P V: B (V tile) MN-major
             const uint32_t tS = tbase + C::S_COL, tO = tbase + C::O_COL;
-            // Two event streams, served as they become ready: S of tile ns (its stage loaded, its S
+            // Two event streams, served as they become ready: S of tile ns (its K half loaded, its S
             // buffer read out by the softmax warps, and for a new pair the queries in shared memory),
-            // and P V of tile npv (its probabilities written).  S thus runs up to two tiles ahead of
-            // the softmax warps.
+            // and P V of tile npv (its probabilities written and its V half loaded).  S thus runs up
+            // to two tiles ahead of the softmax warps.
             int ns = 0, npv = 0, cur_pair = -1, npairs = 0;
             uint32_t first_bits = 0;  // bit t % 32: tile t opens its pair (ns - npv <= NS < 32)
             bool ok = true;
@@ -458,10 +458,11 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
         }
     } else if (warp < nsw) {
         // ================================================================ softmax / epilogue
-        // tcgen05.ld .16x256b on the M = 64 accumulator: thread t of warp w holds query rows
+        // tcgen05.ld .16x256b on the M = 64 accumulator: thread t of warp w holds MMA rows
         // 16 w + t / 4 (h = 0) and 16 w + t / 4 + 8 (h = 1), at columns 8 k + 2 (t % 4) + {0, 1},
-        // k = 0..7 of a 64-column tile: register 4 k + 2 h + e.  Each row is spread over the four
-        // threads with the same t / 4; its maximum and sums combine with two shuffles.
+        // k = 0..7 of a 64-column tile: register 4 k + 2 h + e.  MMA row 16 w + l holds query row
+        // w rpq + l (l < rpq; the others are padding).  Each row is spread over the four threads with
+        // the same t / 4; its maximum and sums combine with two shuffles.
         const int rb = 16 * warp + (lane >> 2);  // MMA row of h = 0; h = 1 is rb + 8
         const int cq = 2 * (lane & 3);           // first column of the thread in each 8-column group
         bool live[2];
