@@ -124,13 +124,20 @@ def draft_window_bytes(cfg, T_list, r, j, W, sink, window):
     return keys * row + 2 * len(T_list) * cfg["Hq"] * cfg["d"] * 2
 
 
-def sources_digest():
-    """sha256 over the code of the library's CUDA sources and C header, comments removed
+# The sources that make each verify kernel (its translation unit, the shared headers and the host
+# code that sizes its launch): an ncu capture stands for that kernel while they hash the same.
+KERNEL_SOURCES = {
+    "ripe_verify_kernel": ("ripe_verify.cu", "ripe_verify.cuh", "ripe_common.cuh"),
+    "ripe_verify_tc_kernel": ("ripe_verify_tc.cu", "ripe_verify.cu", "ripe_verify.cuh", "ripe_common.cuh"),
+}
+
+
+def sources_digest(kernel="ripe_verify_kernel"):
+    """sha256 over the code of a verify kernel's CUDA sources and the C header, comments removed
     (ties an ncu capture to a kernel version)."""
-    import glob
     import hashlib
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "self_speculative_decode_b200", "csrc", "*.cu*")))
+    files = [os.path.join(ROOT, "self_speculative_decode_b200", "csrc", f) for f in KERNEL_SOURCES[kernel]]
     files += [os.path.join(ROOT, "include", "ripe.h")]
     for path in files:
         with open(path, encoding="utf-8") as f:
@@ -148,7 +155,8 @@ def captured_traffic(config):
                 if "=" in line and not line.lstrip().startswith("#"):
                     k, v = line.split("=", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("sources_sha256") != sources_digest() or f"{config}.bytes_per_launch" not in kv:
+        kernel = verify_kernel_name(CONFIGS[config])
+        if kv.get(f"{kernel}.sources_sha256") != sources_digest(kernel) or f"{config}.bytes_per_launch" not in kv:
             return None
         return {"bytes_per_launch": float(kv[f"{config}.bytes_per_launch"]),
                 "T": int(kv[f"{config}.T"]) if f"{config}.T" in kv else None,

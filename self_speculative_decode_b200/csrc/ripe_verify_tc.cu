@@ -24,7 +24,7 @@
 //                                      TMA stage as an MN-major operand)
 //              once the softmax has written P_i (bf16, shared memory) and V_i has landed; each
 //              product frees its half of the stage with tcgen05.commit.
-// The softmax takes two tiles of a (sequence, kv head) at a time and keeps the row's running
+// The softmax takes one tile per iteration (two with RIPE_TC_PAIR) and keeps the row's running
 // maximum m and sums l in registers (base 2).  The maximum moves only when a tile's maximum
 // exceeds it by more than 8 (exact; the rescale of O, a tensor-memory read-modify-write of the
 // thread's row, is then rare).  Rows past the query count are zero in Q and never written out.
@@ -35,6 +35,11 @@
 
 #ifndef RIPE_TC_MAX_STAGES
 #define RIPE_TC_MAX_STAGES 8  // K/V stage cap (shared memory sets the rest)
+#endif
+#ifndef RIPE_TC_PAIR
+// 1: the softmax takes two tiles of a (sequence, kv head) per iteration; 0 (measured faster at 32
+// and 64 query rows: 244 vs 254 us and 297 vs 305 us per long-context call): one
+#define RIPE_TC_PAIR 0
 #endif
 #ifndef RIPE_TC_K_AHEAD
 #define RIPE_TC_K_AHEAD 3     // tiles by which the K loads run ahead of the V loads
@@ -690,15 +695,18 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
                 }
             };
 
-            // Tiles are taken two at a time when both belong to the same (sequence, kv head): their
-            // scores are processed interleaved (instruction-level parallelism for the one warp per
-            // sub-partition) and one lazy-maximum update covers both (an online softmax over a
-            // 128-key block), which also halves the waits and arrivals per tile.
+            // With RIPE_TC_PAIR, tiles are taken two at a time when both belong to the same (sequence,
+            // kv head): their scores are processed interleaved (instruction-level parallelism for the
+            // one warp per sub-partition) and one lazy-maximum update covers both.  Without it (the
+            // default) one tile per iteration, which never waits for the next tile's K.
             int i = 0;
             while (i < ntiles) {
                 const int s0 = i % NS;
                 if (!mbar_wait_bounded(fullK0 + 8 * s0, (i / NS) & 1)) { give_up(); break; }
                 const TileDesc dsc0 = sdesc[s0];
+                // the descriptor is copied: the K half of this tile may be reloaded once S is computed
+                __syncwarp();
+                if (lane == 0) mbar_arrive(emptyK0 + 8 * s0);
                 if (dsc0.pair != cur_pair) {
                     // (a CTA's tiles are consecutive in the concatenated lists: its pairs follow each
                     // other with no gap)
@@ -731,18 +739,14 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
                 }
                 TileDesc dsc1 = dsc0;
                 bool two = false;
-                if (i + 1 < ntiles) {
+                if (RIPE_TC_PAIR && i + 1 < ntiles) {
                     const int s1 = (i + 1) % NS;
                     if (!mbar_wait_bounded(fullK0 + 8 * s1, ((i + 1) / NS) & 1)) { give_up(); break; }
                     dsc1 = sdesc[s1];
                     two = dsc1.pair == dsc0.pair;
-                }
-                // the descriptors are copied: the K halves of the tiles taken may be reloaded once S is
-                // computed (a tile left for the next iteration is read again then)
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(emptyK0 + 8 * s0);
-                    if (two) mbar_arrive(emptyK0 + 8 * ((i + 1) % NS));
+                    // (a tile left for the next iteration releases its K half then)
+                    __syncwarp();
+                    if (two && lane == 0) mbar_arrive(emptyK0 + 8 * s1);
                 }
                 // ---- S of the tile(s): 32 scores each
                 uint32_t sv0[32], sv1[32];
