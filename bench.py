@@ -145,8 +145,10 @@ def sources_digest(kernel="ripe_verify_kernel"):
     return h.hexdigest()
 
 
-def captured_traffic(config):
-    """DRAM bytes per verify launch from the committed ncu summary, if it matches these sources."""
+def captured_traffic(config, kernel=None):
+    """DRAM bytes per verify launch from the committed ncu summary for this workload and kernel (the
+    one the library runs now unless given), if the kernel's sources still hash to the captured ones."""
+    kernel = kernel or verify_kernel_name(CONFIGS[config])
     path = os.path.join(ROOT, "profiles", "ripe_verify_traffic.txt")
     try:
         kv = {}
@@ -155,22 +157,22 @@ def captured_traffic(config):
                 if "=" in line and not line.lstrip().startswith("#"):
                     k, v = line.split("=", 1)
                     kv[k.strip()] = v.strip()
-        kernel = verify_kernel_name(CONFIGS[config])
-        if kv.get(f"{kernel}.sources_sha256") != sources_digest(kernel) or f"{config}.bytes_per_launch" not in kv:
+        key = f"{config}.{kernel}"
+        if kv.get(f"{kernel}.sources_sha256") != sources_digest(kernel) or f"{key}.bytes_per_launch" not in kv:
             return None
-        return {"bytes_per_launch": float(kv[f"{config}.bytes_per_launch"]),
-                "T": int(kv[f"{config}.T"]) if f"{config}.T" in kv else None,
-                "algorithmic_bytes": float(kv[f"{config}.algorithmic_bytes"])
-                if f"{config}.algorithmic_bytes" in kv else None}
+        return {"bytes_per_launch": float(kv[f"{key}.bytes_per_launch"]),
+                "T": int(kv[f"{key}.T"]) if f"{key}.T" in kv else None,
+                "algorithmic_bytes": float(kv[f"{key}.algorithmic_bytes"])
+                if f"{key}.algorithmic_bytes" in kv else None}
     except Exception:
         return None
 
 
-def traffic_for(config, alg_bytes):
+def traffic_for(config, alg_bytes, kernel=None):
     """DRAM bytes per timed verify launch: the captured launch's bytes, scaled by algorithmic bytes
     from the captured launch (the committed prefix length) to the timed ones (a few blocks longer;
     a launch's traffic grows with the key rows it reads)."""
-    t = captured_traffic(config)
+    t = captured_traffic(config, kernel)
     if not t:
         return None
     if t["algorithmic_bytes"]:
@@ -178,21 +180,21 @@ def traffic_for(config, alg_bytes):
     return t["bytes_per_launch"]
 
 
-def traffic_basis(config):
-    t = captured_traffic(config)
+def traffic_basis(config, kernel=None):
+    t = captured_traffic(config, kernel)
     if not t:
-        return "no ncu capture of these sources for this config"
+        return "no ncu capture of these sources for this workload and kernel"
     return (f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at T = {t['T']} (cold L2), "
             "scaled by algorithmic bytes to the timed launches")
 
 
 def verify_kernel_name(cfg):
-    """The verify kernel the library picks for this workload's launches (its default dispatch):
-    the tcgen05 consumer for head_dim 128 with 57..64 query rows per kv head on long pairs."""
+    """The verify kernel that serves this workload's launches: the tcgen05 consumer only when the
+    process selected it (ripe_set_verify_consumer, or RIPE_VERIFY_CONSUMER=tc) and the launch has
+    more than 8 query rows per kv head."""
+    from self_speculative_decode_b200 import ripe
     rows = cfg["B"] * cfg["Hq"] // cfg["kvH"]
-    tiles_per_cta = cfg["N"] * cfg["kvH"] * (cfg["T"] // 64) / 148
-    consumer = os.environ.get("RIPE_VERIFY_CONSUMER")
-    tc = consumer == "tc" and rows > 8 or (consumer != "mma" and cfg["d"] == 128 and rows >= 57 and tiles_per_cta >= 128)
+    tc = rows > 8 and ripe.ripe_get_verify_consumer() == ripe.RIPE_CONSUMER_TC
     return "ripe_verify_tc_kernel" if tc else "ripe_verify_kernel"
 
 
@@ -775,23 +777,34 @@ def huginn_extra(args, device, peak, l2):
 
 
 def gqa64_extra(args, device, peak, l2):
-    """Long-context GQA with 64 query rows per kv head (8 q heads per kv head): the launches the
-    library sends to its tcgen05 consumer.  RIPE layout: the step, each verify launch warm and
-    cold against the roofline, and the wavefront call."""
+    """Long-context GQA with 64 query rows per kv head (8 q heads per kv head), RIPE layout, on each
+    consumer of such launches: the mma.sync kernel (the library's default) and the tcgen05 kernel.
+    Per consumer: the step, each verify launch warm and cold against the roofline, the wavefront call."""
+    from self_speculative_decode_b200 import ripe
     cfg = CONFIGS["gqa64"]
     sub = argparse.Namespace(**vars(args))
-    m = bench_layout(cfg, "ripe", sub, args.seed, device, False, peak, want_extras=False)
-    v = m["verify"]
-    return {"workload": cfg["workload"], "kernel": verify_kernel_name(cfg),
-            "layouts": {"ripe": layout_summary(m, peak)},
+    out = {"workload": cfg["workload"], "consumers": {}}
+    for name, consumer in (("mma", ripe.RIPE_CONSUMER_MMA), ("tc", ripe.RIPE_CONSUMER_TC)):
+        prev = ripe.ripe_set_verify_consumer(consumer)
+        try:
+            kernel = verify_kernel_name(cfg)
+            m = bench_layout(cfg, "ripe", sub, args.seed, device, False, peak, want_extras=False)
+        finally:
+            ripe.ripe_set_verify_consumer(prev)
+        v = m["verify"]
+        out["consumers"][name] = {
+            "kernel": kernel, "layouts": {"ripe": layout_summary(m, peak)},
             "roofline": {"achieved": v["warm"]["gbs"], "frac": v["warm"]["frac"],
                          "launch_us": v["warm"]["us_per_launch"], "bytes_per_launch": v["warm"]["bytes_per_launch"],
-                         "traffic": traffic_for("gqa64", v["warm"]["bytes_per_launch"]),
-                         "traffic_basis": traffic_basis("gqa64")},
+                         "traffic": traffic_for("gqa64", v["warm"]["bytes_per_launch"], kernel),
+                         "traffic_basis": traffic_basis("gqa64", kernel)},
             "roofline_cold": {"achieved": v["cold"]["gbs"], "frac": v["cold"]["frac"],
                               "launch_us": v["cold"]["us_per_launch"]},
-            "l2": l2_note(v["warm"]["bytes_per_launch"], step_distinct_bytes(cfg, v["T"][0], cfg["W"], cfg["L"]), l2),
             "wavefront": {"loops": m["wave"]["loops"], "ripe_us": m["wave"]["us_per_call"], "ripe_gbs": m["wave"]["gbs"]}}
+        out["l2"] = l2_note(v["warm"]["bytes_per_launch"], step_distinct_bytes(cfg, v["T"][0], cfg["W"], cfg["L"]), l2)
+    c = out["consumers"]
+    out["tc_over_mma_launch"] = c["tc"]["roofline"]["launch_us"] / c["mma"]["roofline"]["launch_us"]
+    return out
 
 
 def sweep_extra(args, device, peak):

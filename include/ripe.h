@@ -156,12 +156,8 @@ int ripe_append_block(ripe_cache_t *c, int layer, int r, int B, const void *k, c
  * Work: split-KV over the deepest-plane region and the window ring in one persistent
  * launch; partial results are merged in the same launch, through the shared memory of a
  * 2-CTA cluster when two CTAs share a (sequence, kv head), else through per-call scratch
- * owned by the cache.  The contractions run on mma.sync tensor-core tiles, or on the tcgen05
- * tensor cores (accumulators in tensor memory) for head_dim 128 with 57..64 query rows per kv
- * head when the host copy of the lengths shows at least 128 key tiles per CTA.  The
- * environment variable RIPE_VERIFY_CONSUMER = "tc" or "mma", read once per process, puts one
- * of the two on every launch with 9..64 query rows; the results agree within the bf16 output
- * rounding, not bit for bit.
+ * owned by the cache.  The contractions run on tensor cores: mma.sync tiles, or for 9..64 query
+ * rows per kv head the tcgen05 consumer when ripe_set_verify_consumer selects it.
  */
 int ripe_verify_attn(ripe_cache_t *c, int layer, int r, const void *q, void *out, float *lse,
                      float scale, void *stream);
@@ -308,6 +304,22 @@ int ripe_verify_attn_static(const ripe_cache_view *view, int layer, int r, const
 
 /* How the library was built: RIPE_BUILD_* bits (no device work, no arguments). */
 int ripe_build_info(void);
+
+/* Which tensor-core consumer serves verification launches with 9..64 query rows per kv head
+ * (launches with 1..8 rows, and those that write the draft block, always use mma.sync tiles). */
+enum ripe_verify_consumer {
+    RIPE_CONSUMER_DEFAULT = 0, /* mma.sync tiles: on B200 the faster one at every measured shape */
+    RIPE_CONSUMER_MMA = 1,     /* mma.sync m16n8k16 tiles, accumulators in registers */
+    RIPE_CONSUMER_TC = 2       /* tcgen05 MMAs with accumulators in tensor memory */
+};
+/* Process-wide choice for the launches enqueued after the call (every device, every cache and the
+ * allocation-free entry point).  The initial value comes from the environment variable
+ * RIPE_VERIFY_CONSUMER ("mma" or "tc"; unset or anything else: RIPE_CONSUMER_DEFAULT).
+ * Returns the previous value, or RIPE_EINVAL (nothing changed) for a value outside the enum.
+ * The two consumers agree within the bf16 output rounding, not bit for bit.  No device work. */
+int ripe_set_verify_consumer(int consumer);
+/* The current choice (RIPE_CONSUMER_*; no device work). */
+int ripe_get_verify_consumer(void);
 
 /* Number of kernel launches the library has enqueued since the cache was allocated. */
 int64_t ripe_launch_count(const ripe_cache_t *c);

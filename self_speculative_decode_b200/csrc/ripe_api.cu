@@ -422,4 +422,8 @@ int64_t ripe_launch_count(const ripe_cache_t *c) { return c ? c->launches : -1; 
 
 int ripe_build_info(void) { return kDebug ? RIPE_BUILD_DEBUG : 0; }
 
+int ripe_set_verify_consumer(int consumer) { return ripe::set_verify_consumer(consumer); }
+
+int ripe_get_verify_consumer(void) { return ripe::get_verify_consumer(); }
+
 }  // extern "C"

@@ -471,6 +471,9 @@ int launch_poison(ripe_cache *c, cudaStream_t s);  // debug builds: refill dead 
 // Raise the verify kernels' dynamic shared-memory limit on `device` (which must be current) to
 // what the largest batch needs; once per device, thread-safe.
 int ensure_verify_attributes(int device);
+// ripe_set_verify_consumer: the consumer of verification launches with 9..64 query rows per kv head
+int set_verify_consumer(int consumer);
+int get_verify_consumer();
 
 // Everything one verify launch needs, for callers that own the buffers and the scratch.
 struct RawVerify {

@@ -35,6 +35,7 @@
 //     scratch; the last to arrive (atomic counter, no spinning) merges them.
 //   * Every wait is bounded: on timeout the kernel records RIPE_DEVERR_WAIT_TIMEOUT, drains
 //     its own copies in flight and returns without writing further results.
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -1003,36 +1004,42 @@ static cudaError_t launch_d(int qc, const LaunchTarget &t, int grid, const Verif
     }
 }
 
-// The consumer for 9..64 query rows per kv head.  By default this file's mma.sync kernel, and the
-// tcgen05 kernel (ripe_verify_tc.cu) only where it measured faster on B200: head_dim 128, 57..64
-// query rows per kv head, and long pairs (at least kTcMinTilesPerCta 64-key tiles per CTA, known
-// when the host copy of the lengths is current).  Measured, 8 sequences x 8 kv heads, 64 rows:
-// 32K keys 302 vs 335 us (tcgen05 vs mma.sync), 4K keys 79 vs 73 us; head_dim 96 / 64 at 32K keys
-// 294 vs 282 / 265 vs 224 us; 32 rows, head_dim 128, 32K keys 254 vs 198 us.  The environment
-// variable RIPE_VERIFY_CONSUMER = "tc" or "mma" puts one consumer on all of 9..64 rows (for A/B
-// timing and the tests of both).  Launches that write the draft block (fused append, draft steps)
-// always use this file's kernel.
-constexpr int kTcMinRows = 57;
-constexpr long kTcMinTilesPerCta = 128;
-enum TcPolicy { kTcAuto, kTcAlways, kTcNever };
-static TcPolicy tc_policy() {
-    static const TcPolicy p = [] {
+// The consumer for 9..64 query rows per kv head (ripe_set_verify_consumer).  By default this
+// file's mma.sync kernel: on B200 it measured faster than the tcgen05 kernel (ripe_verify_tc.cu) at
+// every shape tried (8 sequences x 8 kv heads, L2 flushed, per call: 64 rows, head_dim 128, 32K keys
+// 283 vs 297 us; 4K keys 64 vs 76 us; head_dim 96 / 64 at 32K keys 265 vs 293 / 217 vs 266 us; 40
+// rows 281 vs 316 us; 32 rows 193 vs 244 us; 16 rows 188 vs 246 us).  Launches that write the draft
+// block (fused append, draft steps) always use this file's kernel.
+static std::atomic<int> g_consumer{-1};  // -1: not read from the environment yet
+
+static int consumer_choice() {
+    int c = g_consumer.load(std::memory_order_relaxed);
+    if (c < 0) {
         const char *e = std::getenv("RIPE_VERIFY_CONSUMER");
-        if (e && std::strcmp(e, "mma") == 0) return kTcNever;
-        if (e && std::strcmp(e, "tc") == 0) return kTcAlways;
-        return kTcAuto;
-    }();
-    return p;
+        const int env = (e && std::strcmp(e, "mma") == 0) ? RIPE_CONSUMER_MMA
+                        : (e && std::strcmp(e, "tc") == 0) ? RIPE_CONSUMER_TC
+                                                           : RIPE_CONSUMER_DEFAULT;
+        int expected = -1;
+        g_consumer.compare_exchange_strong(expected, env);
+        c = g_consumer.load(std::memory_order_relaxed);
+    }
+    return c;
+}
+
+int get_verify_consumer() { return consumer_choice(); }
+
+int set_verify_consumer(int consumer) {
+    if (consumer < RIPE_CONSUMER_DEFAULT || consumer > RIPE_CONSUMER_TC) return RIPE_EINVAL;
+    const int prev = consumer_choice();
+    g_consumer.store(consumer, std::memory_order_relaxed);
+    return prev;
 }
 
 // tiles: the launch's 64-key tiles when known on the host, else -1
-static cudaError_t launch_any(int d, int qc, const LaunchTarget &t, int grid, const VerifyArgs &a, long tiles,
+static cudaError_t launch_any(int d, int qc, const LaunchTarget &t, int grid, const VerifyArgs &a,
                               cudaStream_t s) {
-    if (qc >= 1 && a.blk_k == nullptr) {
-        const TcPolicy p = tc_policy();
-        const bool tc_auto = d == 128 && a.Mq >= kTcMinRows && tiles >= kTcMinTilesPerCta * grid;
-        if (p == kTcAlways || (p == kTcAuto && tc_auto)) return launch_verify_tc(d, t, grid, a, s);
-    }
+    if (qc >= 1 && a.blk_k == nullptr && consumer_choice() == RIPE_CONSUMER_TC)
+        return launch_verify_tc(d, t, grid, a, s);
     switch (d) {
         case 64: return launch_d<RIPE_QCFG_LIST(64)>(qc, t, grid, a, s);
         case 96: return launch_d<RIPE_QCFG_LIST(96)>(qc, t, grid, a, s);
@@ -1079,7 +1086,7 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.scale_log2 = rv.scale * 1.4426950408889634f;
     const LaunchTarget t = {&rv.tmKd, &rv.tmVd, &rv.tmKw, &rv.tmVw, rv.device, rv.num_sms, rv.N};
     if (rv.d != 64 && rv.d != 96 && rv.d != 128) return RIPE_EINVAL;
-    return launch_any(rv.d, qcfg_of(a.Mq), t, rv.grid, a, -1, s) == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
+    return launch_any(rv.d, qcfg_of(a.Mq), t, rv.grid, a, s) == cudaSuccess ? RIPE_OK : RIPE_ECUDA;
 }
 static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scale, cudaStream_t s);
 
@@ -1182,9 +1189,8 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
 
     // grid: one CTA per SM, fewer when the host copy of T says there is less work
     int grid = c->num_sms < 256 ? c->num_sms : 256;  // the last-CTA merge keeps <= 256 partial weights per row
-    long total = -1;
     if (c->synced) {
-        total = 0;
+        long total = 0;
         for (int n = 0; n < c->N; ++n) total += static_cast<long>(seq_geom(c->T[n], a.plan).total) * c->kvH;
         const long need = (total + a.min_chunk - 1) / a.min_chunk;
         if (need < grid) grid = static_cast<int>(need);
@@ -1192,7 +1198,7 @@ static int launch_cache_args(ripe_cache *c, int layer, VerifyArgs &a, float scal
     if (grid < 1) grid = 1;
     if (c->d != 64 && c->d != 96 && c->d != 128) return RIPE_EINVAL;
     const LaunchTarget t = {&c->tm_Kd, &c->tm_Vd, &c->tm_Kw, &c->tm_Vw, c->device, c->num_sms, c->N};
-    const cudaError_t e = launch_any(c->d, qc, t, grid, a, total, s);
+    const cudaError_t e = launch_any(c->d, qc, t, grid, a, s);
     c->launches += 1;
     c->lengths_dirty = false;
     return e == cudaSuccess ? RIPE_OK : RIPE_ECUDA;

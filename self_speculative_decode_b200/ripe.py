@@ -19,6 +19,7 @@ RIPE_OK, RIPE_EINVAL, RIPE_ENOMEM, RIPE_ECAPACITY, RIPE_ESTATE, RIPE_ECUDA = 0, 
 RIPE_WINDOW_QUERY_RELATIVE, RIPE_WINDOW_CACHE_RELATIVE = 0, 1
 RIPE_DEVERR_WAIT_TIMEOUT, RIPE_DEVERR_CAPACITY, RIPE_DEVERR_ACCEPT, RIPE_DEVERR_BOUNDS = 1, 2, 4, 8
 RIPE_BUILD_DEBUG = 1
+RIPE_CONSUMER_DEFAULT, RIPE_CONSUMER_MMA, RIPE_CONSUMER_TC = 0, 1, 2
 
 # exported entry points (kept in step with include/ripe.h; a CPU test checks both)
 EXPORTS = (
@@ -26,7 +27,8 @@ EXPORTS = (
     "ripe_verify_attn", "ripe_commit", "ripe_commit_device", "ripe_sync_lengths",
     "ripe_cache_stats", "ripe_cache_export", "ripe_get_device_error", "ripe_launch_count",
     "ripe_strerror", "ripe_verify_attn_static", "ripe_verify_attn_wave", "ripe_append_verify",
-    "ripe_draft_attn", "ripe_draft_attn_window", "ripe_build_info",
+    "ripe_draft_attn", "ripe_draft_attn_window", "ripe_build_info", "ripe_set_verify_consumer",
+    "ripe_get_verify_consumer",
 )
 RIPE_ESCRATCH = -6
 RIPE_STATIC_SCRATCH_BYTES = 4 << 20
@@ -80,6 +82,8 @@ def lib() -> ctypes.CDLL:
             "ripe_get_device_error": ([vp, ctypes.POINTER(ctypes.c_uint32), vp], i),
             "ripe_launch_count": ([vp], i64),
             "ripe_build_info": ([], i),
+            "ripe_set_verify_consumer": ([i], i),
+            "ripe_get_verify_consumer": ([], i),
             "ripe_strerror": ([i], ctypes.c_char_p),
             "ripe_verify_attn_static": ([ctypes.POINTER(CacheView), i, i, vp, vp, vp, ctypes.c_float, vp, vp], i),
             "ripe_verify_attn_wave": ([vp, i, i32p, vp, vp, vp, ctypes.c_float, vp], i),
@@ -231,6 +235,18 @@ def ripe_launch_count(h):
 
 def ripe_build_info():
     return lib().ripe_build_info()
+
+
+def ripe_set_verify_consumer(consumer):
+    """Select the consumer of verification launches with 9..64 query rows per kv head (process-wide);
+    returns the previous choice."""
+    prev = lib().ripe_set_verify_consumer(int(consumer))
+    _check(prev if prev < 0 else RIPE_OK, "ripe_set_verify_consumer")
+    return prev
+
+
+def ripe_get_verify_consumer():
+    return lib().ripe_get_verify_consumer()
 
 
 # ------------------------------------------------------------------ tensor-level wrapper

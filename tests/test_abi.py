@@ -67,6 +67,23 @@ def test_calls_on_a_null_handle_are_rejected():
     assert L.ripe_launch_count(null) == -1
 
 
+def test_verify_consumer_selection():
+    """ripe_set_verify_consumer: returns the previous choice, refuses values outside the enum and
+    changes nothing then (no device work: runs without a GPU)."""
+    L = ripe.lib()
+    first = L.ripe_set_verify_consumer(ripe.RIPE_CONSUMER_TC)
+    assert first in (ripe.RIPE_CONSUMER_DEFAULT, ripe.RIPE_CONSUMER_MMA, ripe.RIPE_CONSUMER_TC)
+    assert L.ripe_get_verify_consumer() == ripe.RIPE_CONSUMER_TC
+    assert L.ripe_set_verify_consumer(ripe.RIPE_CONSUMER_MMA) == ripe.RIPE_CONSUMER_TC
+    assert L.ripe_set_verify_consumer(7) == ripe.RIPE_EINVAL
+    assert L.ripe_set_verify_consumer(-1) == ripe.RIPE_EINVAL
+    assert ripe.ripe_get_verify_consumer() == ripe.RIPE_CONSUMER_MMA
+    assert ripe.ripe_set_verify_consumer(first) == ripe.RIPE_CONSUMER_MMA
+    with pytest.raises(ripe.RipeError):
+        ripe.ripe_set_verify_consumer(3)
+    assert L.ripe_set_verify_consumer(first) == first
+
+
 def test_build_info_tells_the_release_and_debug_builds_apart():
     """ripe_build_info: 0 for libripe.so; RIPE_BUILD_DEBUG for libripe_debug.so, which exports the
     same entry points."""

@@ -5,7 +5,7 @@
   against the oracle, and block-split independence checked on the GPU for every W >= B-1;
 * long-context GQA: 32 q / 8 kv heads x 128, R=32, T=32768, W=64, B=8, batch 8, rho 0.85
   (one layer of four), RIPE and full-cache layouts; and the same with 64 q heads (64 query rows
-  per kv head, the tensor-core consumer's launch);
+  per kv head);
 * streaming decode: 16 sequences, Huginn heads, R=32, W=64, B=8, accepted lengths drawn
   U{0..8} per step, fresh drafts every step, from T0=512 and from ragged lengths near 4000
   (where 1000 steps end): verify parity on sampled steps, loops, sequences and heads, and the
@@ -111,8 +111,8 @@ def test_long_context_gqa_sampled(layout, cuda_device):
 
 
 def test_long_context_64_rows_sampled(cuda_device):
-    """64 query rows per kv head (GQA 8, block 8), head_dim 128, 32K keys: the launch the tensor-core
-    consumer serves by default (long pairs, 57..64 rows, head_dim 128)."""
+    """64 query rows per kv head (GQA 8, block 8), head_dim 128, 32K keys (tests/test_gpu_consumers.py
+    reruns it on each consumer)."""
     c = Case(N=8, L=1, Hq=64, kvH=8, d=128, R=4, T=32768, W=64, B=8, rho=0.85, seed=9, backend="torch",
              oracle_seqs=[0, 7], oracle_kvh=[0, 5], oracle_planes={0, 3})
     for r in (0, 3):
