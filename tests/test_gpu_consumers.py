@@ -28,6 +28,7 @@ CASES = [
     "tests/test_gpu_configs.py::test_long_context_64_rows_sampled",
     "tests/test_gpu_wave.py",
     "tests/test_gpu_fused.py::test_fused_append_verify_is_bitwise_the_two_calls",
+    "tests/test_zz_no_alloc.py",
 ]
 
 

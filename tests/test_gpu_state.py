@@ -143,3 +143,62 @@ def test_device_commit_clamps_and_flags_bad_lengths(cuda_device):
     assert gpu.device_error() == ripe.RIPE_DEVERR_ACCEPT
     assert gpu.device_error() == 0                # reading clears the word
     gpu.close()
+
+
+@pytest.mark.parametrize("W", [5, 0, 1000])
+def test_checkpoint_and_resume_through_export_and_load_prefix(W, cuda_device):
+    """A cache's committed state, exported per (sequence, layer) and loaded plane by plane into a fresh
+    cache with ripe_load_prefix, is the same state: equal exports bit for bit, and equal verification
+    results bit for bit on the next block (same kernel, same inputs)."""
+    N, L, kvH, d, R, max_B, max_T = 3, 2, 2, 64, 3, 6, 90
+    rng = np.random.default_rng(29 + W)
+    a_cache = RipeCache(N, L, 2 * kvH, kvH, d, R, W, max_T, max_B)
+    rand = lambda *shape: bits_to_dev((rng.integers(0, 1 << 16, size=shape, dtype=np.uint16) & 0xBFFF).astype(np.uint16),
+                                      cuda_device)
+    T0 = [7, 0, 19]
+    for layer in range(L):
+        for pl in range(R):
+            a_cache.load_prefix(layer, pl, T0, rand(N, kvH, 20, d), rand(N, kvH, 20, d))
+    for step in range(9):   # ragged decode: ring wrap-around and eviction
+        for layer in range(L):
+            for pl in range(R):
+                a_cache.append_block(layer, pl, rand(N, 5, kvH, d), rand(N, 5, kvH, d))
+        a_cache.commit(rng.integers(0, 6, size=N).astype(np.int32))
+    T = a_cache.sync_lengths()
+    # checkpoint: the logical view of every (sequence, layer)
+    views = {(n, layer): a_cache.export(n, layer) for n in range(N) for layer in range(L)}
+    # resume: plane by plane, positions 0 .. T_n - 1 of every sequence
+    b_cache = RipeCache(N, L, 2 * kvH, kvH, d, R, W, max_T, max_B)
+    ld = max(T)
+    for layer in range(L):
+        for pl in range(R):
+            k = torch.zeros((N, kvH, ld, d), dtype=torch.bfloat16, device=cuda_device)
+            v = torch.zeros_like(k)
+            for n in range(N):
+                kx, vx, _ = views[(n, layer)]
+                k[n, :, :T[n]] = kx[pl, :, :T[n]]
+                v[n, :, :T[n]] = vx[pl, :, :T[n]]
+            b_cache.load_prefix(layer, pl, T, k, v)
+    assert b_cache.sync_lengths() == T
+    for n in range(N):
+        for layer in range(L):
+            ka, va, pa = views[(n, layer)]
+            kb, vb, pb = b_cache.export(n, layer)
+            assert torch.equal(pa, pb)
+            assert torch.equal(ka.view(torch.int16), kb.view(torch.int16))
+            assert torch.equal(va.view(torch.int16), vb.view(torch.int16))
+    assert a_cache.stats()["stored_position_planes"] == b_cache.stats()["stored_position_planes"]
+    # the next block on both: the same outputs, bit for bit
+    blk = [(rand(N, 4, kvH, d), rand(N, 4, kvH, d)) for _ in range(L * R)]
+    q = rand(N, 4, 2 * kvH, d)
+    outs = []
+    for c in (a_cache, b_cache):
+        for layer in range(L):
+            for pl in range(R):
+                c.append_block(layer, pl, *blk[layer * R + pl])
+        outs.append([c.verify_attn(layer, r, q).view(torch.int16).clone() for layer in range(L) for r in range(R)])
+    for x, y in zip(*outs):
+        assert torch.equal(x, y)
+    for c in (a_cache, b_cache):
+        assert c.device_error() == 0
+        c.close()
