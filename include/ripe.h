@@ -276,9 +276,10 @@ int ripe_get_device_error(ripe_cache_t *c, uint32_t *err_out, void *stream);
  *
  * The first call on a device sets up that device (looks up the array's device address and
  * the SM count) with the device current; make that first call before any stream capture.
- * Every call shares the array and it keeps the last call's contents; the counters are
- * cleared on `stream` at each call.  Calls that overlap on the GPU (other streams, or other
- * host threads) race on the array and must be serialised by the caller.
+ * Every call shares the array and it keeps the last call's contents; each call tags the
+ * counters with a call number of its own, so nothing is cleared in between (a call that passes
+ * `device_error` enqueues only its kernel).  Calls that overlap on the GPU (other streams, or
+ * other host threads) race on the array and must be serialised by the caller.
  * The view's buffers must stay valid until the work enqueued on `stream` has finished.
  * `device_error` (device uint32, optional) receives RIPE_DEVERR_* bits; the caller clears it.
  * Pass it: with NULL the bits go to a word inside the static array that the next call clears,

@@ -484,6 +484,7 @@ struct RawVerify {
     const int32_t *T;
     float *part_o, *part_ml;
     int32_t *counters;
+    uint32_t epoch;  // nonzero: epoch-tagged arrival counters (no clearing between launches)
     uint32_t *err;
     PlanArgs plan;
     int N, kvH, g, Hq, d, layer, grid, has_deep;

@@ -6,6 +6,7 @@
 // the per-(sequence, kv head) arrival counters -- lives in one file-scope device array of
 // RIPE_STATIC_SCRATCH_BYTES that every GPU loading the library holds until the process exits.
 // The kernel is the same one ripe_verify_attn launches.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -21,6 +22,7 @@ struct DeviceSetup {
     bool done;
     unsigned char *scratch;  // device address of g_static_scratch on this device
     int num_sms;
+    std::atomic<uint32_t> epoch;  // of the last call on this device (tags the arrival counters)
 };
 DeviceSetup g_setup[kMaxDevices];
 std::mutex g_setup_mu;
@@ -180,8 +182,11 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     unsigned char *base = ds->scratch;
     int32_t *counters = reinterpret_cast<int32_t *>(base + off_cnt);
     uint32_t *err = device_error ? device_error : reinterpret_cast<uint32_t *>(base + off_err);
-    // the array keeps the previous call's contents: the counters (and our own error word) start at zero
-    if (cudaMemsetAsync(counters, 0, pairs * sizeof(int32_t), s) != cudaSuccess) return RIPE_ECUDA;
+    // The array keeps the previous call's contents.  The arrival counters need no clearing: each
+    // call tags them with its own epoch (never 0 in the low 16 bits), so whatever an earlier call
+    // left in them counts as zero.  Our own error word starts each call at zero.
+    uint32_t epoch = ds->epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+    if ((epoch & 0xFFFFu) == 0) epoch = ds->epoch.fetch_add(1, std::memory_order_relaxed) + 1;
     if (!device_error && cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess) return RIPE_ECUDA;
 
     rv.q = q;
@@ -191,6 +196,7 @@ extern "C" int ripe_verify_attn_static(const ripe_cache_view *v, int layer, int 
     rv.part_o = reinterpret_cast<float *>(base);
     rv.part_ml = reinterpret_cast<float *>(base + off_ml);
     rv.counters = counters;
+    rv.epoch = epoch;
     rv.err = err;
     rv.plan.W = W;
     rv.plan.B = v->block_len;

@@ -622,8 +622,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
         if (!sole && !abort_now && tid == 0) {
             // publish this CTA's partial (bar.sync + one fence covers every thread's writes)
             __threadfence();
-            const int old = atomicAdd(&a.counters[p], 1);
-            if (old == nparts - 1) {
+            if (arrive_last(&a.counters[p], nparts, a.epoch)) {
                 __threadfence();
                 sflag[4 + sflag[3]] = p;  // merged at the end of this CTA's tiles
                 sflag[3] += 1;
@@ -1057,6 +1056,7 @@ int launch_verify_raw(const RawVerify &rv, cudaStream_t s) {
     a.ring_k = a.ring_v = nullptr;
     a.max_T = 0;
     a.xpair = 0;
+    a.epoch = rv.epoch;
     a.q = static_cast<const __nv_bfloat16 *>(rv.q);
     a.out = static_cast<__nv_bfloat16 *>(rv.out);
     a.lse = rv.lse;
@@ -1095,6 +1095,7 @@ static int launch_single_loop(ripe_cache *c, int layer, int r, int B, int j0, in
                               float *lse, float scale, cudaStream_t s, const void *blk_k, const void *blk_v,
                               int sink = 0, int dwin = -1) {
     VerifyArgs a;
+    a.epoch = 0;
     a.blk_k = static_cast<const uint4 *>(blk_k);
     a.blk_v = static_cast<const uint4 *>(blk_v);
     a.q = static_cast<const __nv_bfloat16 *>(q);
@@ -1134,6 +1135,7 @@ int launch_draft(ripe_cache *c, int layer, int r, int j, const void *k, const vo
 int launch_verify_wave(ripe_cache *c, int layer, const int32_t *loop_of_position, const void *q, void *out,
                        float *lse, float scale, cudaStream_t s) {
     VerifyArgs a;
+    a.epoch = 0;
     a.blk_k = a.blk_v = nullptr;
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.out = static_cast<__nv_bfloat16 *>(out);

@@ -30,6 +30,10 @@ struct VerifyArgs {
     // it (programmatic dependent launch); everything else waits
     int early;
     float scale_log2;
+    // 0: the arrival counters start the launch at zero (the merging CTA clears each after use).
+    // Otherwise the launch's epoch: a counter's top 16 bits tag the launch that last counted on it,
+    // so counters left by an earlier launch count as zero and need no clearing in between.
+    uint32_t epoch;
     // fused append (ripe_append_verify): block K/V [N][B][kvH][d] written to ring plane r
     const uint4 *blk_k, *blk_v;
     uint4 *ring_k, *ring_v;
@@ -57,6 +61,21 @@ constexpr int kSwitchTiles = 3;     // tiles a CTA may add to its chunk to avoid
 struct TileDesc {
     int pair, n, kh, T, kind, t0, cnt, plane;
 };
+
+// One CTA's partial of pair p is published: true for the last of the nparts arrivals (that CTA
+// merges them).  With an epoch (VerifyArgs::epoch) the count lives in the low 16 bits beside the
+// epoch's low 16 bits; a CAS loop that only ever retries after another CTA's arrival succeeded.
+__device__ __forceinline__ bool arrive_last(int32_t *counter, int nparts, uint32_t epoch) {
+    if (epoch == 0) return atomicAdd(counter, 1) == nparts - 1;
+    const uint32_t tag = (epoch & 0xFFFFu) << 16;
+    uint32_t old = *reinterpret_cast<volatile uint32_t *>(counter);
+    for (;;) {
+        const uint32_t cnt = (old & 0xFFFF0000u) == tag ? (old & 0xFFFFu) : 0u;
+        const uint32_t got = atomicCAS(reinterpret_cast<unsigned int *>(counter), old, tag | (cnt + 1));
+        if (got == old) return static_cast<int>(cnt + 1) == nparts;
+        old = got;
+    }
+}
 
 // index of the last sequence whose first tile is <= gt
 __device__ __forceinline__ int seq_of(const int *cum, int N, int gt) {

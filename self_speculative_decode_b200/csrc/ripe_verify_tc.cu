@@ -594,8 +594,7 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
                 epi_sync();  // every row's partial written
                 if (!sole && !abort_now && tid == 0) {
                     __threadfence();
-                    const int old = atomicAdd(&a.counters[p], 1);
-                    if (old == nparts - 1) {
+                    if (arrive_last(&a.counters[p], nparts, a.epoch)) {
                         __threadfence();
                         sflag[4 + sflag[3]] = p;  // merged at the end of this CTA's tiles
                         sflag[3] += 1;
