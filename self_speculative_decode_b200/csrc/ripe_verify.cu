@@ -741,9 +741,12 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                     x[sb][nq][e] = v;
                 }
         }
-        // column maxima over this warp's keys, then over the 8 lanes sharing a column
-        float alpha[NQT][2];
-        bool need = false;
+        // column maxima over this thread's keys; the reference of a column moves only when its
+        // maximum over the warp exceeds the reference by more than kLazyMax, which is so exactly
+        // when one lane's own maximum does.  Only then are the maxima reduced over the 8 lanes
+        // sharing a column (most tiles skip those shuffles, and their exponentials do not wait)
+        float mloc[NQT][2];
+        bool over = false;
 #pragma unroll
         for (int nq = 0; nq < NQT; ++nq)
 #pragma unroll
@@ -751,17 +754,25 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
                 float mt = -INFINITY;
 #pragma unroll
                 for (int sb = 0; sb < C::SB; ++sb) mt = fmaxf(mt, fmaxf(x[sb][nq][e], x[sb][nq][e + 2]));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-                alpha[nq][e] = 1.f;
-                if (mt > m_ref[nq][e] + kLazyMax) {  // also true when m_ref is -inf and mt is finite
-                    alpha[nq][e] = exp2f(m_ref[nq][e] - mt);
-                    m_ref[nq][e] = mt;
-                    need = true;
-                }
+                mloc[nq][e] = mt;
+                over = over || mt > m_ref[nq][e] + kLazyMax;  // also true when m_ref is -inf and mt is finite
             }
-        if (__any_sync(0xffffffffu, need)) {
+        if (__any_sync(0xffffffffu, over)) {
+            float alpha[NQT][2];
+#pragma unroll
+            for (int nq = 0; nq < NQT; ++nq)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float mt = mloc[nq][e];
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+                    alpha[nq][e] = 1.f;
+                    if (mt > m_ref[nq][e] + kLazyMax) {
+                        alpha[nq][e] = exp2f(m_ref[nq][e] - mt);
+                        m_ref[nq][e] = mt;
+                    }
+                }
 #pragma unroll
             for (int nq = 0; nq < NQT; ++nq) {
                 l_run[nq][0] *= alpha[nq][0];

@@ -765,19 +765,29 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
                 float x0[32], x1[32], mt0[2], mt1[2] = {-INFINITY, -INFINITY};
                 scores(dsc0, sv0, x0, mt0);
                 if (two) scores(dsc1, sv1, x1, mt1);
-                float alpha[2] = {1.f, 1.f};
+                // a row's reference moves only when its maximum exceeds it by more than kLazyMax,
+                // which is so exactly when one of the row's four threads sees such a key: only then
+                // are the maxima combined over those threads
+                float alpha[2] = {1.f, 1.f}, mloc[2];
+                bool over = false;
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
-                    float mt = fmaxf(mt0[h], mt1[h]);
-                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-                    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-                    alpha[h] = 1.f;
-                    if (mt > m_ref[h] + kLazyMax) {  // also true when m_ref is -inf and mt is finite
-                        alpha[h] = m_ref[h] == -INFINITY ? 0.f : exp2f(m_ref[h] - mt);
-                        m_ref[h] = mt;
+                    mloc[h] = fmaxf(mt0[h], mt1[h]);
+                    over = over || mloc[h] > m_ref[h] + kLazyMax;  // also true when m_ref is -inf and mt is finite
+                }
+                if (__any_sync(0xffffffffu, over)) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        float mt = mloc[h];
+                        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+                        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+                        if (mt > m_ref[h] + kLazyMax) {
+                            alpha[h] = m_ref[h] == -INFINITY ? 0.f : exp2f(m_ref[h] - mt);
+                            m_ref[h] = mt;
+                        }
+                        l_run[h] *= alpha[h];
+                        l_bf[h] *= alpha[h];
                     }
-                    l_run[h] *= alpha[h];
-                    l_bf[h] *= alpha[h];
                 }
                 uint32_t pk0[16], pk1[16];
                 probs(x0, pk0);
