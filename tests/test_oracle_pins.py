@@ -140,6 +140,38 @@ def test_softmax_weights_sum_to_one():
     assert np.abs(out - 1.0).max() < 1e-12
 
 
+
+def test_zero_scale_is_the_mean_of_the_visible_values():
+    """Scale 0 makes every logit 0: the weights are uniform over keys 0..p, so the output is the
+    plain mean of the values there and the log-sum-exp is ln(p + 1), whichever planes the rule
+    picks when every stored plane of a position holds the same value."""
+    N, kvH, g, d, R, W, T, B = 2, 2, 2, 8, 4, 5, 30, 4
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W, T, B, seed=7, independent=True)
+    q = orc.bf16_to_f64(src.queries(1, B, kvH * g))
+    for r in (0, 1, R - 1):
+        Kr, Vr, Kl, Vl, _ = c.verify_inputs(0, r)
+        X = np.random.default_rng(3).standard_normal(Vr.shape)
+        out, lse = orc.verify(c.T, B, r, R, W, g, Kr, np.where(np.isnan(Vr), np.nan, X),
+                              Kl, np.where(np.isnan(Vl), np.nan, X), q, scale=0.0)
+        for n in range(N):
+            for j in range(B):
+                p = int(c.T[n]) + j
+                for h in range(kvH * g):
+                    assert np.abs(out[n, j, h] - X[n, h // g, :p + 1].mean(axis=0)).max() < 1e-12
+                    assert abs(lse[n, j, h] - np.log(p + 1)) < 1e-12
+
+
+def test_negative_scale_is_attention_with_negated_queries():
+    """softmax(-s <q, k>) = softmax(s <-q, k>): the full cache at scale -0.7 is textbook causal
+    attention (torch SDPA, fp64) of the negated queries at scale 0.7."""
+    N, kvH, g, d, R, T, B = 1, 2, 2, 16, 4, 37, 5
+    c, PK, PV, src = _cache(N, kvH, g, d, R, W=T + B, T=T, B=B, seed=2)
+    for r in (0, 3):
+        q = src.queries(r, B, kvH * g)
+        out, _ = c.verify(0, r, q, g, scale=-0.7)
+        ref = _sdpa(-_f64(q[0]), _f64(PK[r][0]), _f64(PV[r][0]), T, B, g, 0.7)
+        assert np.abs(out[0] - ref).max() < 1e-12
+
 def test_softmax_weights_match_independent_formulations():
     """oracle.weights against two formulations that share none of its code.
 
