@@ -94,7 +94,8 @@ typedef struct ripe_stats {
 } ripe_stats;
 
 /*
- * Allocate a cache for `batch` sequences.
+ * Allocate a cache for `batch` sequences (1 .. 1024: the verify kernels keep every sequence's
+ * length and tile count in shared memory).
  *   layers      recurrent layers L (>= 1)
  *   q_heads     query heads Hq; kv_heads divides it, query head h uses kv head h / (Hq / kv_heads)
  *   head_dim    d, one of 64, 96, 128

@@ -36,6 +36,7 @@ def test_strerror_covers_every_status():
 
 @pytest.mark.parametrize("args", [
     (0, 1, 2, 2, 64, 4, 16, 128, 4, 0),        # no sequences
+    (1025, 1, 2, 2, 64, 4, 16, 128, 4, 0),     # more sequences than the kernels keep in shared memory
     (1, 1, 3, 2, 64, 4, 16, 128, 4, 0),        # q heads not a multiple of kv heads
     (1, 1, 2, 2, 80, 4, 16, 128, 4, 0),        # unsupported head_dim
     (1, 1, 2, 2, 64, 0, 16, 128, 4, 0),        # no loops

@@ -197,6 +197,8 @@ def test_streaming_decode_late_lengths(cuda_device):
     dict(N=2, L=1, Hq=4, kvH=4, d=96, R=1, T=[500, 77], W=16, B=8),          # one loop: ordinary attention
     dict(N=2, L=1, Hq=64, kvH=8, d=128, R=3, T=[700, 64], W=20, B=8),        # 64 query rows per kv head
     dict(N=1, L=1, Hq=2, kvH=1, d=64, R=2, T=[63], W=63, B=1),               # a single key tile, W = T
+    dict(N=1024, L=1, Hq=2, kvH=1, d=64, R=2, T=[(37 * n) % 97 for n in range(1024)], W=8, B=2),
+    # the largest batch a cache takes, ragged lengths 0..96
 ])
 def test_edge_shapes(kw, cuda_device):
     c = Case(**kw, seed=9, independent=True)

@@ -63,6 +63,18 @@ def test_large_logit_scale(cuda_device):
     c.close()
 
 
+
+@pytest.mark.parametrize("g,B", [(1, 8), (4, 8)])
+def test_degenerate_logit_scales(g, B, cuda_device):
+    """Scale 0 (uniform weights over the visible keys: every tile's logits tie) and negative scales
+    (the largest logit comes from the smallest score), on 8 and 32 query rows per kv head."""
+    c = Case(N=2, L=1, Hq=2 * g, kvH=2, d=128, R=3, T=[300, 77], W=20, B=B, seed=6, independent=True)
+    for r in range(3):
+        for scale in (0.0, -1.0, -8.0):
+            c.check(0, r, scale=scale)
+    c.close()
+
+
 @pytest.mark.parametrize("layout", ["full", "ripe", "deepest"])
 def test_huginn_shape(layout, cuda_device):
     """4 recurrent layers, 55 MHA heads x 96, R=32, T=1024, W=64, B=8, batch 1, rho 0.88."""
