@@ -74,3 +74,34 @@ def test_l2_note_classifies_working_sets():
     cfg = dict(N=1, kvH=55, d=96, R=32, B=8)
     row = 4 * 55 * 96
     assert bench.step_distinct_bytes(cfg, 1024, 64, 4) == 4 * row * (960 + 32 * 72)
+
+
+def test_captured_traffic_stands_only_for_the_sources_it_hashes(tmp_path, monkeypatch):
+    """A committed ncu capture is used while the kernel's sources hash to the recorded digest and is
+    scaled by algorithmic bytes to the timed launch; once the sources change the bench reports no
+    traffic rather than a stale figure."""
+    f = tmp_path / "ripe_verify_traffic.txt"
+    f.write_text("# header\n"
+                 f"ripe_verify_kernel.sources_sha256 = {bench.sources_digest('ripe_verify_kernel')}\n"
+                 "long_gqa.ripe_verify_kernel.bytes_per_launch = 1010\n"
+                 "long_gqa.ripe_verify_kernel.T = 32768\n"
+                 "long_gqa.ripe_verify_kernel.algorithmic_bytes = 1000\n")
+    real_join = bench.os.path.join
+    monkeypatch.setattr(bench.os.path, "join",
+                        lambda *p: str(f) if p[-1] == "ripe_verify_traffic.txt" else real_join(*p))
+    k = "ripe_verify_kernel"
+    assert bench.captured_traffic("long_gqa", k) == {"bytes_per_launch": 1010.0, "T": 32768,
+                                                     "algorithmic_bytes": 1000.0}
+    assert bench.traffic_for("long_gqa", 2000, k) == 2020.0           # scaled by algorithmic bytes
+    assert bench.captured_traffic("huginn", k) is None                 # no capture of that workload
+    monkeypatch.setattr(bench, "sources_digest", lambda kernel="ripe_verify_kernel": "0" * 64)
+    assert bench.captured_traffic("long_gqa", k) is None               # the sources changed
+    assert bench.traffic_for("long_gqa", 2000, k) is None
+    assert bench.traffic_basis("long_gqa", k).startswith("no ncu capture")
+
+
+def test_sources_digest_ignores_comments_only():
+    """Comment and blank-line edits keep a capture valid; a change of code does not."""
+    code = "int f(int a) {\n  return a + 1;  // one more\n}\n"
+    assert bench._code_only(code) == bench._code_only("/* doc */\nint f(int a) {\n\n  return a + 1;\n}\n")
+    assert bench._code_only(code) != bench._code_only(code.replace("a + 1", "a + 2"))
