@@ -11,6 +11,10 @@ compared with the pairs the queries of the block select under the RIPE rule (ora
     row at that loop sees); a pair is read twice only at the deepest plane, when the call includes
     the deepest loop (its ring tiles and the older window keys then cover the same rows; the masks
     give each query one of them);
+  * a draft step (one query at block position j, optionally restricted to an attention sink and a
+    sliding window) reads every pair its query selects; of the deepest-plane region it reads
+    exactly the selected rows (a windowed draft skips the rows between the sink and the window),
+    and beyond that only the ring at its loop and the older window keys at the deepest plane;
   * every tile is one box of consecutive rows: deepest-plane rows at row t, ring rows at slot
     t mod S, never across the ring's wrap, never past the committed positions and the block.
 """
@@ -41,7 +45,9 @@ def dump(tmp_path_factory):
                    check=True, capture_output=True, timeout=600)
 
     def run(cases):
-        text = "".join(" ".join(str(x) for x in (*c[:7], len(c[7]), *c[7])) + "\n" for c in cases)
+        lines = [" ".join(str(x) for x in c) if c[0] == "D" else
+                 " ".join(str(x) for x in ("V", *c[:7], len(c[7]), *c[7])) for c in cases]
+        text = "\n".join(lines) + "\n"
         out = subprocess.run([exe], input=text, capture_output=True, text=True, check=True, timeout=120).stdout
         plans, cur = [], []
         for line in out.splitlines():
@@ -136,3 +142,30 @@ def test_wavefront_plan_covers_every_row_at_its_loop(dump):
         for (t, plane), k in got.items():
             if k > 1:
                 assert k == 2 and plane == R - 1 and R - 1 in loop_of_j and t < T, (case, t)
+
+
+def test_draft_step_plans(dump):
+    rng = np.random.default_rng(13)
+    cases = []
+    for _ in range(400):
+        R = int(rng.choice([1, 2, 5, 32]))
+        T = int(rng.choice([0, 1, 5, 64, 65, 200, int(rng.integers(0, 600))]))
+        W = int(rng.choice([0, 1, 4, 8, 64, 300, 5000]))
+        max_B = int(rng.integers(1, 17))
+        j = int(rng.integers(0, max_B))
+        max_T = T + max_B + int(rng.choice([0, 3, 100]))
+        window = int(rng.choice([-1, 0, 1, 7, 64, 100, 1000]))
+        sink = int(rng.choice([0, 1, 4, 70])) if window >= 0 else 0
+        cases.append(("D", T, W, R, max_T, max_B, int(rng.integers(0, 2)), int(rng.integers(0, R)), j, sink, window))
+    for case, tiles in zip(cases, dump(cases)):
+        _, T, W, R, max_T, max_B, mode, r, j, sink, window = case
+        Wc, S = _geometry(W, max_T, max_B)
+        got = _read(T, j + 1, Wc, S, tiles)
+        p = T + j
+        keep = [t for t in range(p + 1) if window < 0 or t < sink or t >= p - window]
+        need = {(t, orc.plane_of(p, t, r, R, T, Wc, mode)) for t in keep}
+        assert need <= set(got), case
+        D = max(0, T - Wc)
+        assert {(t, pl) for (t, pl) in got if t < D} == {(t, pl) for (t, pl) in need if t < D}, case
+        allowed = {(t, r) for t in range(D, p + 1)} | {(t, R - 1) for t in range(D, T)}
+        assert set(got) - need <= allowed, case

@@ -1,22 +1,35 @@
 // Host-only dump of the tile list that the verify kernels walk for one (sequence, kv head), with
-// the plan set up as the library's launch code sets it up (ripe_verify.cu: launch_single_loop and
-// launch_verify_wave).  tests/test_tile_plan.py compiles it with nvcc and checks the tiles against
+// the plan set up as the library's launch code sets it up (ripe_verify.cu: launch_single_loop,
+// launch_draft and launch_verify_wave).  tests/test_tile_plan.py compiles it with nvcc and checks the tiles against
 // the oracle's plane rule; nothing here runs on a GPU.
 //
-// Input, one case per line:  T W B R max_T max_B mode nloops loop_0 .. loop_{nloops-1}
-//   (nloops = 1: a single-loop verification at loop_0; nloops > 1: a wavefront call whose block
-//    position j sits at loop_{j mod nloops})
+// Input, one case per line:
+//   V T W B R max_T max_B mode nloops loop_0 .. loop_{nloops-1}
+//     verification (nloops = 1: one call at loop_0; nloops > 1: a wavefront call whose block
+//     position j sits at loop_{j mod nloops})
+//   D T W R max_T max_B mode r j sink window
+//     a draft step at block position j and loop r (launch_draft: the plan's block is positions
+//     0..j, the query is position j; window = -1 for a full-context draft)
 // Output per case: one line "kind t0 cnt y plane" per tile, then "E total".
 #include <cstdio>
 
 #include "ripe_common.cuh"
 
 int main() {
-    int T, W, B, R, max_T, max_B, mode, nloops;
-    while (std::scanf("%d %d %d %d %d %d %d %d", &T, &W, &B, &R, &max_T, &max_B, &mode, &nloops) == 8) {
+    char what[4];
+    while (std::scanf("%3s", what) == 1) {
+        int T, W, B, R, max_T, max_B, mode, nloops = 1, sink = 0, dwin = -1, dj = 0;
         int loops[ripe::kMaxQueryRows];
-        for (int k = 0; k < nloops; ++k)
-            if (std::scanf("%d", &loops[k]) != 1) return 2;
+        if (what[0] == 'V') {
+            if (std::scanf("%d %d %d %d %d %d %d %d", &T, &W, &B, &R, &max_T, &max_B, &mode, &nloops) != 8) return 2;
+            for (int k = 0; k < nloops; ++k)
+                if (std::scanf("%d", &loops[k]) != 1) return 2;
+        } else {
+            if (std::scanf("%d %d %d %d %d %d %d %d %d %d", &T, &W, &R, &max_T, &max_B, &mode, &loops[0], &dj, &sink,
+                           &dwin) != 10)
+                return 2;
+            B = dj + 1;
+        }
         // cache geometry (ripe_cache_alloc)
         const int Wc = W > max_T ? max_T : W;
         const int ring_slots = Wc + max_B < max_T ? Wc + max_B : max_T;
@@ -28,9 +41,9 @@ int main() {
         pa.ring_slots = ring_slots;
         pa.deep_box = (deep_rows == 0 || deep_rows >= ripe::kTileRows) ? ripe::kTileRows : deep_rows;
         pa.ring_box = ring_slots < ripe::kTileRows ? ring_slots : ripe::kTileRows;
-        pa.sink = 0;
-        pa.dwin = -1;
-        pa.dj = 0;
+        pa.sink = sink;
+        pa.dwin = dwin;
+        pa.dj = dj;
         if (nloops == 1) {  // single loop: at the deepest loop the window rule changes nothing
             pa.mode_eff = (mode == RIPE_WINDOW_CACHE_RELATIVE || loops[0] == R - 1) ? 1 : 0;
             pa.nloops = 1;
