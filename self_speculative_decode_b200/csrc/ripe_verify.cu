@@ -755,7 +755,7 @@ ripe_verify_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_consta
 #pragma unroll
                 for (int sb = 0; sb < C::SB; ++sb) mt = fmaxf(mt, fmaxf(x[sb][nq][e], x[sb][nq][e + 2]));
                 mloc[nq][e] = mt;
-                over = over || mt > m_ref[nq][e] + kLazyMax;  // also true when m_ref is -inf and mt is finite
+                over = over || mt > m_ref[nq][e] + kLazyMax;  // also true for a finite maximum when m_ref is -inf
             }
         if (__any_sync(0xffffffffu, over)) {
             float alpha[NQT][2];

@@ -773,7 +773,7 @@ ripe_verify_tc_kernel(const __grid_constant__ CUtensorMap tmKd, const __grid_con
 #pragma unroll
                 for (int h = 0; h < NH; ++h) {
                     mloc[h] = fmaxf(mt0[h], mt1[h]);
-                    over = over || mloc[h] > m_ref[h] + kLazyMax;  // also true when m_ref is -inf and mt is finite
+                    over = over || mloc[h] > m_ref[h] + kLazyMax;  // also true for a finite maximum when m_ref is -inf
                 }
                 if (__any_sync(0xffffffffu, over)) {
 #pragma unroll
